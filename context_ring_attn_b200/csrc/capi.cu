@@ -1,0 +1,404 @@
+// Device entry points of libcpattn.so: argument checks, work tables, tensor
+// maps and kernel launches. Every check happens before the first launch; the
+// library allocates nothing and keeps no state beyond a cached driver entry
+// point.
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "cp_attn.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "merge.cuh"
+#include "partial_simt.cuh"
+#include "partial_tc.cuh"
+#include "work.cuh"
+
+namespace {
+
+using namespace cpk;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+inline int ilog2_exact(int x) {
+  int l = 0;
+  while ((1 << l) < x) ++l;
+  return ((1 << l) == x) ? l : -1;
+}
+
+cp_status last_cuda_status() { return cudaGetLastError() == cudaSuccess ? CP_OK : CP_ERR_CUDA; }
+
+bool range_ok(const cp_range& r) { return r.len >= 0 && r.row0 >= 0 && r.pos0 >= 0 && r.reserved == 0; }
+
+// ---------------------------------------------------------------------------
+// work tables
+// ---------------------------------------------------------------------------
+struct SegSort {
+  WorkSeg seg;
+  int64_t cost;  // visible keys of the segment's most expensive tile
+};
+
+// Split the blocks into launches whose tables fit the kernel parameter space.
+// Within a launch, segments run longest-first so the tail of the grid holds
+// the cheap tiles.
+bool build_tables(const cp_range* ranges, const cp_block* blocks, int32_t n_blocks, int tok_per_tile, int causal,
+                  std::vector<WorkTable>& tables) {
+  tables.clear();
+  std::vector<SegSort> segs;
+  std::vector<int32_t> local;  // global range index -> local index, -1 if absent
+  std::vector<cp_range> lranges;
+  std::vector<int32_t> touched;
+
+  auto flush = [&]() {
+    if (segs.empty()) return;
+    std::stable_sort(segs.begin(), segs.end(), [](const SegSort& a, const SegSort& b) { return a.cost > b.cost; });
+    tables.emplace_back();
+    WorkTable& wt = tables.back();
+    std::memset(&wt, 0, sizeof(WorkTable));
+    wt.n_segs = static_cast<int32_t>(segs.size());
+    int32_t acc = 0;
+    for (size_t i = 0; i < segs.size(); ++i) {
+      wt.segs[i] = segs[i].seg;
+      wt.tile_prefix[i] = acc;
+      acc += segs[i].seg.n_tiles;
+    }
+    wt.tile_prefix[segs.size()] = acc;
+    wt.total_tiles = acc;
+    std::copy(lranges.begin(), lranges.end(), wt.ranges);
+    segs.clear();
+    lranges.clear();
+    for (int32_t g : touched) local[g] = -1;
+    touched.clear();
+  };
+
+  int32_t max_index = 0;
+  for (int32_t b = 0; b < n_blocks; ++b)
+    max_index = std::max(max_index, std::max(blocks[b].q_begin + blocks[b].q_count, blocks[b].kv_begin + blocks[b].kv_count));
+  local.assign(max_index + 1, -1);
+
+  for (int32_t b = 0; b < n_blocks; ++b) {
+    const cp_block& bl = blocks[b];
+    if (bl.q_count > kMaxSegs || bl.q_count + bl.kv_count > kMaxRanges) return false;
+    // ranges this block needs that the current table lacks
+    int need = 0;
+    for (int32_t j = 0; j < bl.q_count; ++j) need += local[bl.q_begin + j] < 0;
+    bool kv_contiguous = true;
+    for (int32_t j = 0; j < bl.kv_count; ++j) {
+      const int32_t g = bl.kv_begin + j;
+      if (local[g] < 0) ++need;
+      else if (j > 0 && local[g] != local[g - 1] + 1) kv_contiguous = false;
+    }
+    if (!kv_contiguous) need += bl.kv_count;  // KV slice is re-added contiguously
+    if (static_cast<int>(lranges.size()) + need > kMaxRanges || static_cast<int>(segs.size()) + bl.q_count > kMaxSegs)
+      flush();
+    // KV slice: contiguous in the local table
+    int32_t kv_local = -1;
+    {
+      bool have = bl.kv_count > 0 && local[bl.kv_begin] >= 0;
+      for (int32_t j = 1; j < bl.kv_count && have; ++j)
+        have = local[bl.kv_begin + j] == local[bl.kv_begin] + j;
+      if (have) {
+        kv_local = local[bl.kv_begin];
+      } else {
+        kv_local = static_cast<int32_t>(lranges.size());
+        for (int32_t j = 0; j < bl.kv_count; ++j) {
+          const int32_t g = bl.kv_begin + j;
+          lranges.push_back(ranges[g]);
+          if (local[g] < 0) touched.push_back(g);
+          local[g] = kv_local + j;
+        }
+      }
+    }
+    for (int32_t j = 0; j < bl.q_count; ++j) {
+      const int32_t g = bl.q_begin + j;
+      const cp_range& qr = ranges[g];
+      if (qr.len == 0) continue;
+      int32_t ql = local[g];
+      if (ql < 0) {
+        ql = static_cast<int32_t>(lranges.size());
+        lranges.push_back(qr);
+        local[g] = ql;
+        touched.push_back(g);
+      }
+      const int64_t n_tiles = (qr.len + tok_per_tile - 1) / tok_per_tile;
+      int64_t cost = 0;
+      for (int32_t r = 0; r < bl.kv_count; ++r) {
+        const cp_range& kr = ranges[bl.kv_begin + r];
+        if (kr.seq == qr.seq) cost += visible_keys(kr, qr.pos0 + qr.len - 1, causal);
+      }
+      SegSort s;
+      s.seg.q_range = ql;
+      s.seg.kv_begin = kv_local;
+      s.seg.kv_count = bl.kv_count;
+      s.seg.n_tiles = static_cast<int32_t>(n_tiles);
+      s.seg.out_row0 = bl.out_row0;
+      s.cost = cost;
+      segs.push_back(s);
+    }
+  }
+  flush();
+  return true;
+}
+
+// Tensor maps: Q as [rows][N_KV][G][D] (box 64 x G x 1 x 128/G), K and V as
+// [rows][N_KV][D] (box 64 x 1 x 128), bf16, 128-byte swizzle.
+bool make_qkv_maps(tc::Params& p, const void* q, const void* k, const void* v, int64_t q_rows, int64_t kv_rows,
+                   int n_h, int n_kv, int group) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint32_t estr4[4] = {1, 1, 1, 1};
+  {
+    const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(group), static_cast<cuuint64_t>(n_kv),
+                                static_cast<cuuint64_t>(q_rows)};
+    const cuuint64_t strides[3] = {128 * 2, static_cast<cuuint64_t>(group) * 256,
+                                   static_cast<cuuint64_t>(n_h) * 256};
+    const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(group), 1, static_cast<cuuint32_t>(128 / group)};
+    if (enc(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(q), dims, strides, box, estr4,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(n_kv), static_cast<cuuint64_t>(kv_rows)};
+  const cuuint64_t strides[2] = {128 * 2, static_cast<cuuint64_t>(n_kv) * 256};
+  const cuuint32_t box[3] = {64, 1, 128};
+  const void* src[2] = {k, v};
+  CUtensorMap* dst[2] = {&p.tm_k, &p.tm_v};
+  for (int i = 0; i < 2; ++i) {
+    if (enc(dst[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(src[i]), dims, strides, box, estr4,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  return true;
+}
+
+constexpr size_t kStatusBytes = 256;
+
+inline size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+extern "C" {
+
+size_t cp_workspace_size(cp_op op, int64_t rows, int32_t n_h, int32_t d, int32_t n_splits) {
+  if (op == CP_OP_DECODE) {
+    if (rows < 0 || n_h < 1 || d < 1 || n_splits < 1) return kStatusBytes;
+    const size_t part = static_cast<size_t>(n_splits) * static_cast<size_t>(rows) * static_cast<size_t>(n_h);
+    return kStatusBytes + round256(part * static_cast<size_t>(d) * 4) + round256(part * 4);
+  }
+  return kStatusBytes;
+}
+
+cp_status cp_reset_status(void* workspace, void* cuda_stream) {
+  if (!workspace) return CP_ERR_WORKSPACE;
+  if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+    return CP_ERR_CUDA;
+  return CP_OK;
+}
+
+cp_status cp_check_status(const void* workspace, void* cuda_stream) {
+  if (!workspace) return CP_ERR_WORKSPACE;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess) return CP_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return CP_ERR_CUDA;
+  if (word & kStatusTimeout) return CP_ERR_TIMEOUT;
+  if (word & kStatusInternal) return CP_ERR_INTERNAL;
+  return CP_OK;
+}
+
+cp_status cp_attn_partial(const void* q, const void* k, const void* v, cp_dtype dtype, int64_t q_rows,
+                          int64_t kv_rows, int32_t n_h, int32_t n_kv, int32_t d, float softmax_scale, int32_t causal,
+                          const cp_range* ranges, int32_t n_ranges, const cp_block* blocks, int32_t n_blocks,
+                          float* o_part, float* lse_part, int64_t out_rows, void* workspace, size_t ws_bytes,
+                          void* cuda_stream) {
+  // ---- arguments
+  if (!q || !k || !v || !o_part || !lse_part) return CP_ERR_INVALID_ARG;
+  if (n_blocks < 0 || n_ranges < 0 || (n_blocks > 0 && (!ranges || !blocks))) return CP_ERR_INVALID_ARG;
+  if (n_h < 1 || n_kv < 1 || d < 1 || q_rows < 0 || kv_rows < 0 || out_rows < 0) return CP_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.0f) || !(softmax_scale < INFINITY)) return CP_ERR_INVALID_ARG;
+  if (n_h % n_kv != 0) return CP_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < kStatusBytes || !aligned(workspace, 256)) return CP_ERR_WORKSPACE;
+  const int group = n_h / n_kv;
+  if (dtype == CP_BF16) {
+    if (d != 128 || ilog2_exact(group) < 0 || group > 128) return CP_ERR_UNSUPPORTED;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return CP_ERR_INVALID_ARG;
+    if (q_rows >= (int64_t(1) << 31) || kv_rows >= (int64_t(1) << 31)) return CP_ERR_UNSUPPORTED;
+  } else if (dtype == CP_F32) {
+    if ((d != 64 && d != 128) || group > simt::kRows) return CP_ERR_UNSUPPORTED;
+    if (!aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4)) return CP_ERR_INVALID_ARG;
+  } else {
+    return CP_ERR_UNSUPPORTED;
+  }
+  if (!aligned(o_part, 16) || !aligned(lse_part, 4)) return CP_ERR_INVALID_ARG;
+  for (int32_t b = 0; b < n_blocks; ++b) {
+    const cp_block& bl = blocks[b];
+    if (bl.q_begin < 0 || bl.q_count < 0 || bl.kv_begin < 0 || bl.kv_count < 0) return CP_ERR_INVALID_ARG;
+    if (int64_t(bl.q_begin) + bl.q_count > n_ranges || int64_t(bl.kv_begin) + bl.kv_count > n_ranges)
+      return CP_ERR_INVALID_ARG;
+    for (int32_t j = 0; j < bl.q_count; ++j) {
+      const cp_range& r = ranges[bl.q_begin + j];
+      if (!range_ok(r) || r.row0 + r.len > q_rows) return CP_ERR_INVALID_ARG;
+      if (r.len > 0 && (bl.out_row0 + r.row0 < 0 || bl.out_row0 + r.row0 + r.len > out_rows)) return CP_ERR_INVALID_ARG;
+    }
+    for (int32_t j = 0; j < bl.kv_count; ++j) {
+      const cp_range& r = ranges[bl.kv_begin + j];
+      if (!range_ok(r) || r.row0 + r.len > kv_rows) return CP_ERR_INVALID_ARG;
+    }
+  }
+  const int tok_per_tile = (dtype == CP_BF16) ? 128 / group : simt::kRows / group;
+  std::vector<WorkTable> tables;
+  if (!build_tables(ranges, blocks, n_blocks, tok_per_tile, causal != 0, tables)) return CP_ERR_UNSUPPORTED;
+
+  int64_t total_tiles = 0;
+  for (const WorkTable& wt : tables) total_tiles += wt.total_tiles;
+  if (total_tiles == 0) return CP_OK;
+
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  const float log2e = 1.4426950408889634f;
+
+  if (dtype == CP_BF16) {
+    static tc::Params params;  // large: kept off the stack; copied at launch
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!make_qkv_maps(params, q, k, v, q_rows, kv_rows, n_h, n_kv, group)) return CP_ERR_CUDA;
+    params.o_part = o_part;
+    params.lse_part = lse_part;
+    params.status = status;
+    params.n_h = n_h;
+    params.log2_group = ilog2_exact(group);
+    params.causal = causal != 0;
+    params.scale_log2 = softmax_scale * log2e;
+    if (cudaFuncSetAttribute(tc::partial_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tc::kSmemBytes) != cudaSuccess)
+      return CP_ERR_CUDA;
+    for (const WorkTable& wt : tables) {
+      if (wt.total_tiles == 0) continue;
+      std::memcpy(&params.wt, &wt, sizeof(WorkTable));
+      dim3 grid(wt.total_tiles, n_kv);
+      tc::partial_bf16_kernel<<<grid, tc::kThreads, tc::kSmemBytes, stream>>>(params);
+      if (last_cuda_status() != CP_OK) return CP_ERR_CUDA;
+    }
+  } else {
+    static simt::Params params;
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    params.q = static_cast<const float*>(q);
+    params.k = static_cast<const float*>(k);
+    params.v = static_cast<const float*>(v);
+    params.o_part = o_part;
+    params.lse_part = lse_part;
+    params.n_h = n_h;
+    params.n_kv = n_kv;
+    params.group = group;
+    params.tok_per_tile = tok_per_tile;
+    params.causal = causal != 0;
+    params.scale = softmax_scale;
+    for (const WorkTable& wt : tables) {
+      if (wt.total_tiles == 0) continue;
+      std::memcpy(&params.wt, &wt, sizeof(WorkTable));
+      dim3 grid(wt.total_tiles, n_kv);
+      if (d == 64)
+        simt::partial_f32_kernel<64><<<grid, simt::kThreads, 0, stream>>>(params);
+      else
+        simt::partial_f32_kernel<128><<<grid, simt::kThreads, 0, stream>>>(params);
+      if (last_cuda_status() != CP_OK) return CP_ERR_CUDA;
+    }
+  }
+  return CP_OK;
+}
+
+cp_status cp_attn_merge(const float* o_parts, const float* lse_parts, int32_t n_parts, int64_t part_stride_rows,
+                        int64_t rows, int32_t n_h, int32_t d, void* out, cp_dtype out_dtype, float* lse_out,
+                        void* cuda_stream) {
+  if (!o_parts || !lse_parts || !out) return CP_ERR_INVALID_ARG;
+  if (n_parts < 1 || rows < 0 || n_h < 1 || d < 4 || (d & 3)) return CP_ERR_INVALID_ARG;
+  if (n_parts > 1 && part_stride_rows < rows) return CP_ERR_INVALID_ARG;
+  if (!aligned(o_parts, 16) || !aligned(lse_parts, 4)) return CP_ERR_INVALID_ARG;
+  if (out_dtype == CP_F32) {
+    if (!aligned(out, 16)) return CP_ERR_INVALID_ARG;
+  } else if (out_dtype == CP_BF16) {
+    if (!aligned(out, 8)) return CP_ERR_INVALID_ARG;
+  } else {
+    return CP_ERR_UNSUPPORTED;
+  }
+  const int64_t n_rowheads = rows * n_h;
+  if (n_rowheads == 0) return CP_OK;
+  const int64_t warps_per_block = merge::kThreads / 32;
+  int64_t grid = (n_rowheads + warps_per_block - 1) / warps_per_block;
+  grid = std::min<int64_t>(grid, 148 * 32);
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  const int64_t o_stride = part_stride_rows * n_h * d;
+  const int64_t l_stride = part_stride_rows * n_h;
+  if (out_dtype == CP_F32)
+    merge::merge_kernel<float><<<static_cast<unsigned>(grid), merge::kThreads, 0, stream>>>(
+        o_parts, lse_parts, n_parts, o_stride, l_stride, n_rowheads, d, static_cast<float*>(out), lse_out);
+  else
+    merge::merge_kernel<__nv_bfloat16><<<static_cast<unsigned>(grid), merge::kThreads, 0, stream>>>(
+        o_parts, lse_parts, n_parts, o_stride, l_stride, n_rowheads, d, static_cast<__nv_bfloat16*>(out), lse_out);
+  return last_cuda_status();
+}
+
+cp_status cp_decode(const void* q, const void* k, const void* v, cp_dtype dtype, const int64_t* kv_offsets,
+                    int32_t batch, int64_t kv_rows, int32_t n_h, int32_t n_kv, int32_t d, int32_t n_splits,
+                    float softmax_scale, void* out, float* lse_out, void* workspace, size_t ws_bytes,
+                    void* cuda_stream) {
+  if (!q || !k || !v || !kv_offsets || !out) return CP_ERR_INVALID_ARG;
+  if (batch < 0 || kv_rows < 0 || n_h < 1 || n_kv < 1 || d < 1 || n_h % n_kv) return CP_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.0f) || !(softmax_scale < INFINITY)) return CP_ERR_INVALID_ARG;
+  if (n_splits < 1 || n_splits > dec::kMaxSplits) return CP_ERR_UNSUPPORTED;
+  const int group = n_h / n_kv;
+  if (dtype != CP_BF16 || d != 128 || group > 16 || (16 % group) != 0) return CP_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 8) || !aligned(kv_offsets, 8))
+    return CP_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < cp_workspace_size(CP_OP_DECODE, batch, n_h, d, n_splits))
+    return CP_ERR_WORKSPACE;
+  if (batch == 0) return CP_OK;
+  const size_t part = static_cast<size_t>(n_splits) * batch * n_h;
+  float* o_ws = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
+  float* l_ws = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes + round256(part * d * 4));
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  dec::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.offsets = kv_offsets;
+  p.kv_rows = kv_rows;
+  p.o_part = o_ws;
+  p.lse_part = l_ws;
+  p.status = static_cast<uint32_t*>(workspace);
+  p.batch = batch;
+  p.n_h = n_h;
+  p.n_kv = n_kv;
+  p.group = group;
+  p.n_splits = n_splits;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  if (cudaFuncSetAttribute(dec::decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           dec::kSmemBytes) != cudaSuccess)
+    return CP_ERR_CUDA;
+  dim3 grid(n_splits, batch * n_kv);
+  dec::decode_split_kernel<<<grid, dec::kThreads, dec::kSmemBytes, stream>>>(p);
+  if (last_cuda_status() != CP_OK) return CP_ERR_CUDA;
+  return cp_attn_merge(o_ws, l_ws, n_splits, batch, batch, n_h, d, out, CP_BF16, lse_out, cuda_stream);
+}
+
+}  // extern "C"

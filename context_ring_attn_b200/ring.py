@@ -1,0 +1,107 @@
+"""Ring schedules over the C ABI: N virtual context-parallel ranks on one GPU.
+
+"Context Parallelism for Scalable Million-Token Inference", section 3: in
+pass-KV every rank keeps its query shard while the KV shards travel around
+the ring; in pass-Q the KV shards stay and the query shards travel, and an
+all-to-all returns the partials to their owners, which merge them. On one
+GPU every shard already sits in the same buffers, so a ring step is one
+cp_attn_partial launch covering the N blocks of that step, and the exchange
+moves no bytes. The merge is cp_attn_merge.
+
+This module only sequences C-ABI calls; all arithmetic runs in the kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from dataclasses import dataclass
+
+import torch
+
+from . import binding as B
+
+
+@dataclass
+class Segment:
+    """`length` rows of a buffer from `row0`, tokens of sequence `seq` at
+    positions pos0.. (a persistent-KV prefill has a cached segment and a new
+    one in the same sequence)."""
+    length: int
+    row0: int
+    pos0: int
+    seq: int = 0
+
+
+class RingSchedule:
+    def __init__(self, q_segs, kv_segs, n_ranks: int, variant: int = B.CP_PASS_KV,
+                 mode: int = B.CP_SHARD_LOAD_BALANCED):
+        self.n_ranks = n_ranks
+        self.variant = variant
+        self.mode = mode
+        self.q_segs = B.segments([(s.length, s.row0, s.pos0, s.seq) for s in q_segs])
+        self.kv_segs = B.segments([(s.length, s.row0, s.pos0, s.seq) for s in kv_segs])
+        self.ranges, self.n_ranges, self.blocks, self.parts = B.cp_ring_schedule(
+            self.q_segs, len(q_segs), self.kv_segs, len(kv_segs), n_ranks, mode, variant)
+
+    def step_blocks(self, t: int, part_rows: int, part_of=None) -> ctypes.Array:
+        """The N blocks of ring step t, writing partial `part_of(part)` at row
+        offset part * part_rows of one stacked partial buffer."""
+        n = self.n_ranks
+        arr = (B.cp_block * n)()
+        for i in range(n):
+            src = self.blocks[t * n + i]
+            part = self.parts[t * n + i] if part_of is None else part_of(self.parts[t * n + i])
+            arr[i] = B.cp_block(src.q_begin, src.q_count, src.kv_begin, src.kv_count, part * part_rows)
+        return arr
+
+    def pairs(self, causal: bool = True) -> int:
+        """Visible (query, key) pairs per query head over the whole schedule."""
+        return sum(B.cp_block_pairs(self.ranges, self.blocks[i], causal) for i in range(self.n_ranks ** 2))
+
+
+def partial_buffers(q_rows: int, n_h: int, d: int, n_parts: int, device="cuda"):
+    o = torch.empty((n_parts * q_rows, n_h, d), dtype=torch.float32, device=device)
+    lse = torch.empty((n_parts * q_rows, n_h), dtype=torch.float32, device=device)
+    return o, lse
+
+
+def run_ring(sched: RingSchedule, q, k, v, n_h: int, n_kv: int, out, lse_out=None, causal: bool = True,
+             scale: float | None = None, o_parts=None, lse_parts=None, workspace=None,
+             merge: str = "final", stream=None):
+    """Attention of q against k/v through the ring schedule, into `out`.
+
+    merge="final": N partial buffers, one N-way merge at the end.
+    merge="running": two partial buffers; after every step the step's partial
+    is merged into the running one (less memory, N-1 extra merge passes).
+    """
+    q_rows, d = int(q.shape[0]), int(q.shape[-1])
+    n = sched.n_ranks
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    n_bufs = n if merge == "final" else 2
+    if o_parts is None:
+        o_parts, lse_parts = partial_buffers(q_rows, n_h, d, n_bufs, q.device)
+    if workspace is None:
+        workspace = torch.zeros(B.cp_workspace_size(B.CP_OP_PARTIAL, 0, n_h, d, 1), dtype=torch.uint8,
+                                device=q.device)
+    if merge == "final":
+        for t in range(n):
+            blocks = sched.step_blocks(t, q_rows)
+            B.cp_attn_partial(q, k, v, n_h, n_kv, scale, causal, sched.ranges, sched.n_ranges, blocks, n,
+                              o_parts, lse_parts, workspace, stream)
+        B.cp_attn_merge(o_parts, lse_parts, n, q_rows, q_rows, n_h, d, out, lse_out, stream)
+    elif merge == "running":
+        for t in range(n):
+            target = 0 if t == 0 else 1
+            blocks = sched.step_blocks(t, q_rows, part_of=lambda _p, _t=target: _t)
+            B.cp_attn_partial(q, k, v, n_h, n_kv, scale, causal, sched.ranges, sched.n_ranges, blocks, n,
+                              o_parts, lse_parts, workspace, stream)
+            if t == 0 and n > 1:
+                continue
+            if t == n - 1:
+                B.cp_attn_merge(o_parts, lse_parts, 2 if n > 1 else 1, q_rows, q_rows, n_h, d, out, lse_out, stream)
+            else:
+                B.cp_attn_merge(o_parts, lse_parts, 2, q_rows, q_rows, n_h, d, o_parts, lse_parts, stream)
+    else:
+        raise ValueError(merge)
+    return out

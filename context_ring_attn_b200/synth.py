@@ -20,6 +20,8 @@ Shapes follow "Context Parallelism for Scalable Million-Token Inference"
 from __future__ import annotations
 
 import itertools
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -63,27 +65,57 @@ def _block_rng(seed: int, tensor_id: int, block: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, tensor_id, block])))
 
 
-def normal_rows(seed: int, tensor_id: int, n_rows: int, row_shape: tuple, std: float,
-                rows: np.ndarray | None = None) -> np.ndarray:
-    """float32 normal tensor [n_rows, *row_shape] (or only ``rows`` of it)."""
+def _threads() -> int:
+    return max(1, min(32, os.cpu_count() or 1))
+
+
+def _blocked(seed, tensor_id, n_rows, row_shape, std, rows, transform, out_dtype):
     width = int(np.prod(row_shape))
     if rows is None:
-        out = np.empty((n_rows, width), dtype=np.float32)
-        for b0 in range(0, n_rows, ROW_BLOCK):
-            nb = min(ROW_BLOCK, n_rows - b0)
-            g = _block_rng(seed, tensor_id, b0 // ROW_BLOCK)
-            out[b0:b0 + nb] = g.standard_normal((ROW_BLOCK, width), dtype=np.float32)[:nb]
-        out *= np.float32(std)
-        return out.reshape((n_rows,) + tuple(row_shape))
-    rows = np.asarray(rows, dtype=np.int64)
-    out = np.empty((rows.size, width), dtype=np.float32)
-    for blk in np.unique(rows // ROW_BLOCK):
+        rows = np.arange(n_rows, dtype=np.int64)
+        contiguous = True
+    else:
+        rows = np.asarray(rows, dtype=np.int64)
+        contiguous = False
+    out = np.empty((rows.size, width), dtype=out_dtype)
+    blocks = np.unique(rows // ROW_BLOCK)
+
+    def fill(blk):
         g = _block_rng(seed, tensor_id, int(blk))
         full = g.standard_normal((ROW_BLOCK, width), dtype=np.float32)
-        sel = np.nonzero(rows // ROW_BLOCK == blk)[0]
-        out[sel] = full[rows[sel] - blk * ROW_BLOCK]
-    out *= np.float32(std)
+        full *= np.float32(std)
+        if contiguous:
+            r0 = int(blk) * ROW_BLOCK
+            nb = min(ROW_BLOCK, n_rows - r0)
+            out[r0:r0 + nb] = transform(full[:nb])
+        else:
+            sel = np.nonzero(rows // ROW_BLOCK == blk)[0]
+            out[sel] = transform(full[rows[sel] - blk * ROW_BLOCK])
+
+    if len(blocks) > 1:
+        with ThreadPoolExecutor(max_workers=_threads()) as ex:
+            list(ex.map(fill, blocks))
+    else:
+        for blk in blocks:
+            fill(blk)
     return out.reshape((rows.size,) + tuple(row_shape))
+
+
+def normal_rows(seed: int, tensor_id: int, n_rows: int, row_shape: tuple, std: float,
+                rows: np.ndarray | None = None) -> np.ndarray:
+    """float32 normal tensor [n_rows, *row_shape] (or only ``rows`` of it).
+
+    Blocks are drawn on a thread pool (each block has its own generator, so
+    the values do not depend on the thread count)."""
+    return _blocked(seed, tensor_id, n_rows, row_shape, std, rows, lambda x: x, np.float32)
+
+
+def raw_rows(seed: int, tensor_id: int, n_rows: int, row_shape: tuple, std: float, dtype: str,
+             rows: np.ndarray | None = None) -> np.ndarray:
+    """The stored form of normal_rows: float32, or bf16 bit patterns (uint16)."""
+    if dtype == "f32":
+        return normal_rows(seed, tensor_id, n_rows, row_shape, std, rows)
+    return _blocked(seed, tensor_id, n_rows, row_shape, std, rows, bf16_bits, np.uint16)
 
 
 def stored_values(x32: np.ndarray, dtype: str) -> tuple[np.ndarray, np.ndarray]:
@@ -191,3 +223,23 @@ WORKLOADS = {
     "varlen_prefill": dict(total=262144, n_seq=8, n_h=128, n_kv=8, d=128, dtype="bf16", seed=1005,
                            std=0.5, n_ranks=8),
 }
+
+
+# --------------------------------------------------------------------------
+# device upload (chunked: a full-size Q never exists in fp32 on the host)
+# --------------------------------------------------------------------------
+def device_rows(seed: int, tensor_id: int, n_rows: int, row_shape: tuple, std: float, dtype: str,
+                device="cuda"):
+    """Generate a tensor block by block and copy each block to the device.
+    Returns a torch tensor [n_rows, *row_shape] of bf16 or fp32."""
+    import torch
+
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    out = torch.empty((n_rows,) + tuple(row_shape), dtype=tdt, device=device)
+    step = ROW_BLOCK * 64
+    for r0 in range(0, n_rows, step):
+        r1 = min(n_rows, r0 + step)
+        raw = raw_rows(seed, tensor_id, n_rows, row_shape, std, dtype, np.arange(r0, r1))
+        src = torch.from_numpy(raw.view(np.int16)).view(torch.bfloat16) if dtype == "bf16" else torch.from_numpy(raw)
+        out[r0:r1].copy_(src)
+    return out

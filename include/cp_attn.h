@@ -1,0 +1,237 @@
+/*
+ * cp_attn.h -- C ABI of libcpattn.so: the hot path of context-parallel ring
+ * attention on one B200 (sm_100a), with the N context-parallel ranks as
+ * virtual shards of one GPU's buffers.
+ *
+ * Method: "Context Parallelism for Scalable Million-Token Inference" (review of
+ * arXiv:2411.01783). Exact GQA softmax attention is computed as partial blocks
+ * (one query shard against one KV shard, online softmax over KV tiles), each
+ * yielding an output normalised within the block plus a per-row log-sum-exp,
+ * and the partials are combined by LSE weighting ("merge attention").
+ *
+ * Conventions shared by every entry point:
+ *  - The caller owns and allocates every buffer. The library never allocates,
+ *    frees or keeps device memory and holds no state between calls.
+ *  - Tensors are row-major and token-major: Q [rows, N_H, D], K and V
+ *    [rows, N_KV, D], partial outputs [rows, N_H, D] fp32, LSE [rows, N_H] fp32
+ *    (natural logarithm of the sum of exp(scaled scores)).
+ *  - Device entry points are asynchronous on the given CUDA stream
+ *    (a cudaStream_t passed as void*, NULL = legacy default stream). They
+ *    validate every argument before launching anything and return a status;
+ *    they never abort or print. A launch failure maps to CP_ERR_CUDA. A fault
+ *    inside a kernel surfaces at the caller's next synchronisation.
+ *  - Device-side waits are bounded. A wait that runs out writes a code into the
+ *    status word at the start of the workspace and the kernel returns early;
+ *    cp_check_status() reports it.
+ *  - Host planning entry points are deterministic and bit-exact.
+ */
+#ifndef CP_ATTN_H
+#define CP_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CP_ABI_VERSION 1
+
+typedef enum {
+  CP_OK = 0,
+  CP_ERR_INVALID_ARG = 1,  /* null pointer, negative size, range outside a buffer */
+  CP_ERR_UNSUPPORTED = 2,  /* valid but not implemented: head dim, dtype, group size */
+  CP_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or too small */
+  CP_ERR_CUDA = 4,         /* a CUDA runtime or driver call failed */
+  CP_ERR_TIMEOUT = 5,      /* a device-side wait ran out (see cp_check_status) */
+  CP_ERR_INTERNAL = 6      /* a device-side consistency check failed */
+} cp_status;
+
+typedef enum { CP_F32 = 0, CP_BF16 = 1 } cp_dtype;
+
+/* Load-balanced: a segment of length L is cut into 2N chunks,
+ * chunk c = [floor(c*L/2N), floor((c+1)*L/2N)), and rank i holds chunks i and
+ * 2N-1-i (method page, section 4, load-balanced sharding).
+ * Contiguous: rank i holds chunks 2i and 2i+1, i.e. [floor(iL/N), floor((i+1)L/N)). */
+typedef enum { CP_SHARD_LOAD_BALANCED = 0, CP_SHARD_CONTIGUOUS = 1 } cp_shard_mode;
+
+/* Ring variants (method page, section 3). Rank r sends to r+1, so at step t
+ * rank r holds the visiting shard of rank (r - t) mod N.
+ *  pass-KV: rank i keeps its Q shard and sees the KV shard of (i - t) mod N;
+ *           that block's partial is arrival number t.
+ *  pass-Q:  rank i keeps its KV shard and sees the Q shard of (i - t) mod N;
+ *           after the all-to-all the Q owner holds one partial per KV owner,
+ *           indexed by the KV owner i. */
+typedef enum { CP_PASS_KV = 0, CP_PASS_Q = 1 } cp_ring_variant;
+
+typedef enum { CP_PAIR_FULL = 0, CP_PAIR_PARTIAL = 1, CP_PAIR_SKIP = 2 } cp_pair_class;
+
+/* A sharding unit: `len` consecutive rows of a buffer starting at `row0`,
+ * holding tokens of sequence `seq` at global positions pos0..pos0+len-1.
+ * A persistent-KV prefill describes the cached prefix and the new tokens as
+ * two segments of the same sequence, each sharded on its own. */
+typedef struct {
+  int64_t len;
+  int64_t row0;
+  int64_t pos0;
+  int32_t seq;
+  int32_t reserved; /* must be 0 */
+} cp_segment;
+
+/* A contiguous run of rows of one buffer (a chunk of a shard). 32 bytes. */
+typedef struct {
+  int64_t row0; /* first row in the Q (or K/V) buffer */
+  int64_t pos0; /* global causal position of that row */
+  int64_t len;  /* number of rows */
+  int32_t seq;  /* sequence id: attention never crosses sequences */
+  int32_t reserved; /* must be 0 */
+} cp_range;
+
+/* One block of the ring: the query ranges ranges[q_begin .. q_begin+q_count)
+ * against the key/value ranges ranges[kv_begin .. kv_begin+kv_count).
+ * Query row r of the Q buffer writes output row out_row0 + r. 24 bytes. */
+typedef struct {
+  int32_t q_begin, q_count;
+  int32_t kv_begin, kv_count;
+  int64_t out_row0;
+} cp_block;
+
+typedef enum { CP_OP_PARTIAL = 0, CP_OP_DECODE = 1, CP_OP_MERGE = 2 } cp_op;
+
+const char* cp_status_string(cp_status s);
+int32_t cp_abi_version(void);
+
+/* ---------------------------------------------------------------------------
+ * Host planning (method page, sections 3 and 4). No device work.
+ * ------------------------------------------------------------------------- */
+
+/* Shard plan of `n_seg` segments over `n_ranks` ranks.
+ *  chunk_bounds [n_seg][2N+1]: per segment, chunk boundaries relative to the
+ *                segment start (floor(c*len/2N)).
+ *  rank_rows    [N+1]: prefix offsets of each rank's rows in token_index.
+ *  token_index  [sum of len]: buffer rows held by rank 0, then rank 1, ...;
+ *                per rank, segment by segment, chunks in ascending order.
+ * Any output pointer may be NULL to skip it. Errors: CP_ERR_INVALID_ARG for
+ * n_ranks < 1, n_seg < 0, a negative len/row0/pos0 or a nonzero reserved field. */
+cp_status cp_shard_plan(const cp_segment* segs, int32_t n_seg, int32_t n_ranks,
+                        cp_shard_mode mode, int64_t* chunk_bounds, int64_t* rank_rows,
+                        int64_t* token_index);
+
+/* The ranges rank `rank` holds: for each segment in order, its two chunks in
+ * ascending chunk order, empty chunks left out. `out` holds up to 2*n_seg
+ * entries; *n_out receives the count. */
+cp_status cp_rank_ranges(const cp_segment* segs, int32_t n_seg, int32_t n_ranks,
+                         cp_shard_mode mode, int32_t rank, cp_range* out, int32_t* n_out);
+
+/* Full ring schedule. ranges receives the Q shards of ranks 0..N-1 followed by
+ * the KV shards of ranks 0..N-1 (at most 2*N*(n_q_seg+n_kv_seg) entries;
+ * `ranges_cap` is the capacity, *n_ranges the count). blocks [N*N]:
+ * blocks[t*N + i] is the block rank i computes at ring step t, with
+ * out_row0 = 0; block_part [N*N] (may be NULL) is the index (0..N-1) of the
+ * partial that block produces for its query rows (see cp_ring_variant). */
+cp_status cp_ring_schedule(const cp_segment* q_segs, int32_t n_q_seg,
+                           const cp_segment* kv_segs, int32_t n_kv_seg, int32_t n_ranks,
+                           cp_shard_mode mode, cp_ring_variant variant, cp_range* ranges,
+                           int32_t ranges_cap, int32_t* n_ranges, cp_block* blocks,
+                           int32_t* block_part);
+
+/* FULL: every query row of q sees every key of kv; PARTIAL: a mask is needed;
+ * SKIP: no pair is visible (other sequence, or every key after every query
+ * when causal). Causal visibility: key position <= query position. */
+cp_pair_class cp_classify_pair(const cp_range* q, const cp_range* kv, int32_t causal);
+
+/* Number of (query, key) pairs of a block that the mask keeps, per query head. */
+int64_t cp_block_pairs(const cp_range* ranges, const cp_block* block, int32_t causal);
+
+/* Elements a real ring would move (the virtual ring moves none). hop_elems
+ * [(N-1)*N]: at hop t (1..N-1), what rank i receives, at [(t-1)*N + i]:
+ * pass-KV counts one KV tensor (K or V), rows*N_KV*D; pass-Q counts the Q
+ * shard, rows*N_H*D. *total sums hop_elems; *all_to_all counts pass-Q's
+ * return of partials, rows*N_H*(D+1) per non-local block (0 for pass-KV).
+ * Any output may be NULL. */
+cp_status cp_ring_comm_volume(const cp_range* ranges, const cp_block* blocks, int32_t n_ranks,
+                              cp_ring_variant variant, int32_t n_h, int32_t n_kv, int32_t d,
+                              int64_t* hop_elems, int64_t* total, int64_t* all_to_all);
+
+/* ---------------------------------------------------------------------------
+ * Device entry points (sm_100a). Pointers named q/k/v/o/lse/out/workspace are
+ * device pointers; ranges/blocks are host arrays read during the call.
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of workspace an entry point needs (always a multiple of 256).
+ *  CP_OP_PARTIAL, CP_OP_MERGE: 256 (the status word).
+ *  CP_OP_DECODE: 256 + the split partials, n_splits*batch*n_h*(d+1)*4 rounded
+ *  up to 256. `rows` is the batch for decode. */
+size_t cp_workspace_size(cp_op op, int64_t rows, int32_t n_h, int32_t d, int32_t n_splits);
+
+/* Zero the status word of a workspace (stream-ordered). */
+cp_status cp_reset_status(void* workspace, void* cuda_stream);
+
+/* Synchronise `cuda_stream` and report the status word of `workspace`:
+ * CP_OK, CP_ERR_TIMEOUT or CP_ERR_INTERNAL. */
+cp_status cp_check_status(const void* workspace, void* cuda_stream);
+
+/* Partial attention of every block (method page, section 3: ring pass-KV and
+ * pass-Q; shapes from section 3, core formulas). For block b, query row r of
+ * range ranges[j] (j in the block's query slice), at position
+ * pos_r = ranges[j].pos0 + (r - ranges[j].row0), and query head h, the visible
+ * keys are the rows of the block's KV ranges of the same sequence with
+ * position <= pos_r (all positions when causal == 0); KV head
+ * g = floor(h / (n_h / n_kv)). Writes, at output row out_row0 + r:
+ *   lse_part[row, h] = ln sum_visible exp(scale * <q, k>)   (-inf if none)
+ *   o_part[row, h, :] = sum_visible exp(scale*<q,k> - lse) * v   (0 if none)
+ * Rows of the output not named by any block are left untouched. Blocks must
+ * not write the same output row twice.
+ *
+ * dtype CP_BF16: tensor-core path (tcgen05/TMEM/TMA), fp32 accumulation,
+ *   probabilities rounded to bf16 before the PV product; needs d == 128,
+ *   n_h % n_kv == 0, the group size n_h/n_kv a power of two <= 128, and
+ *   16-byte aligned q/k/v.
+ * dtype CP_F32: exact fp32 SIMT path; d in {64, 128}.
+ * q_rows / kv_rows / out_rows: rows allocated in q, k/v and o_part/lse_part;
+ * every range must lie inside its buffer (CP_ERR_INVALID_ARG otherwise).
+ * workspace: >= cp_workspace_size(CP_OP_PARTIAL, ...) bytes, 256-byte aligned. */
+cp_status cp_attn_partial(const void* q, const void* k, const void* v, cp_dtype dtype,
+                          int64_t q_rows, int64_t kv_rows, int32_t n_h, int32_t n_kv, int32_t d,
+                          float softmax_scale, int32_t causal, const cp_range* ranges,
+                          int32_t n_ranges, const cp_block* blocks, int32_t n_blocks,
+                          float* o_part, float* lse_part, int64_t out_rows, void* workspace,
+                          size_t ws_bytes, void* cuda_stream);
+
+/* LSE merge of n_parts partials of the same rows (method page, section 5,
+ * implementation detail 3: the merge after pass-Q; the same step closes
+ * pass-KV). Part j lives at o_parts + j*part_stride_rows*n_h*d and
+ * lse_parts + j*part_stride_rows*n_h. Per (row, head):
+ *   M = max_j lse_j;  lse = M + ln sum_j exp(lse_j - M);
+ *   out = sum_j exp(lse_j - lse) * o_j.
+ * Parts with lse = -inf get weight 0; if all are -inf, out = 0 and lse = -inf.
+ * out [rows, n_h, d] is written as out_dtype (bf16: round to nearest even);
+ * lse_out [rows, n_h] may be NULL. With out_dtype CP_F32, out may be the
+ * same buffer as part 0 (and lse_out as lse part 0): each element is read
+ * before it is written, by the same thread. Requires d % 4 == 0 and 16-byte
+ * aligned o_parts/out. */
+cp_status cp_attn_merge(const float* o_parts, const float* lse_parts, int32_t n_parts,
+                        int64_t part_stride_rows, int64_t rows, int32_t n_h, int32_t d, void* out,
+                        cp_dtype out_dtype, float* lse_out, void* cuda_stream);
+
+/* Split-KV decode (Flash Decoding with n_splits splits per request; method
+ * page, section 5 software stack). Request b has one query row q[b] at
+ * position L_b - 1 and keys k/v rows kv_offsets[b] .. kv_offsets[b+1]-1
+ * (L_b = difference), all visible. Split s covers request keys
+ * [floor(s*L_b/n_splits), floor((s+1)*L_b/n_splits)); each split's partial
+ * goes to the workspace, then the splits are merged as in cp_attn_merge.
+ *   q [batch, n_h, d] bf16; k, v [kv_rows, n_kv, d] bf16;
+ *   kv_offsets: DEVICE int64 [batch+1], non-decreasing, last <= kv_rows;
+ *   out [batch, n_h, d] bf16; lse_out [batch, n_h] fp32 (may be NULL).
+ * Supports dtype CP_BF16, d == 128, n_h/n_kv == 16, 1 <= n_splits <= 1024.
+ * A request with L_b = 0 yields out = 0, lse = -inf.
+ * workspace: >= cp_workspace_size(CP_OP_DECODE, batch, n_h, d, n_splits). */
+cp_status cp_decode(const void* q, const void* k, const void* v, cp_dtype dtype,
+                    const int64_t* kv_offsets, int32_t batch, int64_t kv_rows, int32_t n_h,
+                    int32_t n_kv, int32_t d, int32_t n_splits, float softmax_scale, void* out,
+                    float* lse_out, void* workspace, size_t ws_bytes, void* cuda_stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CP_ATTN_H */

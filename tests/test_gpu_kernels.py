@@ -1,0 +1,195 @@
+"""GPU parity of each kernel against the fp64 reference on small seeded
+inputs that still span several tiles and a ragged tail."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from context_ring_attn_b200 import binding as B
+from context_ring_attn_b200 import ring, synth
+from oracle import attention as OA
+from oracle import decode as OD
+from oracle import plan as OP
+
+from gpu_util import check, dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    B.lib()
+
+
+def _ws():
+    return torch.zeros(256, dtype=torch.uint8, device="cuda")
+
+
+def _run_prefill(pr, n_ranks, variant, mode, merge="final", q_scale=1.0, segs=None):
+    """Ring attention through the library vs the unsharded reference."""
+    t, p = pr.t, pr.p
+    q_np = pr.q * q_scale
+    q_raw = synth.bf16_bits(q_np) if pr.dtype == "bf16" else q_np.astype(np.float32)
+    q = dev(q_raw, pr.dtype)
+    k, v = dev(pr.k_raw, pr.dtype), dev(pr.v_raw, pr.dtype)
+    if segs is None:
+        q_segs = [ring.Segment(t, 0, p, 0)]
+        kv_segs = [ring.Segment(p, 0, 0, 0), ring.Segment(t, p, p, 0)] if p else [ring.Segment(t, 0, 0, 0)]
+        q_pos, k_pos = np.arange(p, p + t), np.arange(p + t)
+        q_seq = k_seq = None
+    else:
+        q_segs = kv_segs = segs
+        q_pos = k_pos = np.concatenate([np.arange(s.pos0, s.pos0 + s.length) for s in segs])
+        q_seq = k_seq = np.concatenate([np.full(s.length, s.seq) for s in segs])
+    sched = ring.RingSchedule(q_segs, kv_segs, n_ranks, variant, mode)
+    out_dt = torch.bfloat16 if pr.dtype == "bf16" else torch.float32
+    out = torch.empty((t, pr.n_h, pr.d), dtype=out_dt, device="cuda")
+    lse = torch.empty((t, pr.n_h), dtype=torch.float32, device="cuda")
+    ring.run_ring(sched, q, k, v, pr.n_h, pr.n_kv, out, lse, merge=merge, workspace=_ws())
+    torch.cuda.synchronize()
+    q_vals = synth.bf16_bits_to_f32(q_raw) if pr.dtype == "bf16" else q_raw
+    o_ref, l_ref = OA.attention(q_vals, pr.k, pr.v, q_pos, k_pos, q_seq, k_seq)
+    return check(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, pr.dtype,
+                 f"{pr.dtype} T={t} P={p} N={n_ranks} var={variant} mode={mode}")
+
+
+# ---------------------------------------------------------------------------- fp32 exact path
+@pytest.mark.parametrize("variant", [B.CP_PASS_KV, B.CP_PASS_Q])
+@pytest.mark.parametrize("mode", [B.CP_SHARD_LOAD_BALANCED, B.CP_SHARD_CONTIGUOUS])
+def test_tiny_exact_fp32(variant, mode):
+    w = synth.WORKLOADS["tiny_exact"]
+    pr = synth.make_prefill(w["t"], w["n_h"], w["n_kv"], w["d"], "f32", w["seed"], w["std"])
+    _run_prefill(pr, w["n_ranks"], variant, mode)
+
+
+@pytest.mark.parametrize("merge", ["final", "running"])
+def test_fp32_gqa_ragged(merge):
+    pr = synth.make_prefill(301, 8, 2, 128, "f32", 11, 1.0, p=77)
+    _run_prefill(pr, 3, B.CP_PASS_Q, B.CP_SHARD_LOAD_BALANCED, merge=merge)
+
+
+def test_fp32_partial_empty_rows_and_noncausal():
+    """A block whose queries sit before part of the KV range: some rows see
+    nothing (O = 0, LSE = -inf); the non-causal block sees everything."""
+    rng = np.random.default_rng(3)
+    n_h, n_kv, d = 4, 2, 64
+    q = rng.standard_normal((50, n_h, d)).astype(np.float32)
+    k = rng.standard_normal((300, n_kv, d)).astype(np.float32)
+    v = rng.standard_normal((300, n_kv, d)).astype(np.float32)
+    ranges = (B.cp_range * 3)(B.cp_range(0, 100, 50, 0, 0), B.cp_range(20, 120, 200, 0, 0),
+                              B.cp_range(0, 100, 20, 0, 0))
+    for causal, blk in ((True, B.cp_block(0, 1, 1, 1, 0)), (False, B.cp_block(0, 1, 1, 2, 0))):
+        blocks = (B.cp_block * 1)(blk)
+        o = torch.full((50, n_h, d), float("nan"), device="cuda")
+        lse = torch.full((50, n_h), float("nan"), device="cuda")
+        B.cp_attn_partial(dev(q, "f32"), dev(k, "f32"), dev(v, "f32"), n_h, n_kv, 1 / 8, causal, ranges, 3,
+                          blocks, 1, o, lse, _ws())
+        torch.cuda.synchronize()
+        kv_rows = np.arange(20, 220) if causal else np.concatenate([np.arange(20, 220), np.arange(0, 20)])
+        k_pos = np.concatenate([np.arange(120, 320), np.arange(100, 120)])[:len(kv_rows)]
+        o_ref, l_ref = OA.attention(q, k[kv_rows], v[kv_rows], np.arange(100, 150), k_pos, scale=1 / 8,
+                                    causal=causal)
+        check(o.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "f32", f"causal={causal}")
+        if causal:
+            assert np.all(np.isinf(l_ref[:20]))
+
+
+# ---------------------------------------------------------------------------- bf16 tensor-core path
+@pytest.mark.parametrize("t,n_h,n_kv,n_ranks,variant,mode", [
+    (1000, 16, 1, 3, B.CP_PASS_KV, B.CP_SHARD_LOAD_BALANCED),
+    (777, 8, 2, 2, B.CP_PASS_Q, B.CP_SHARD_LOAD_BALANCED),
+    (1024, 16, 1, 4, B.CP_PASS_KV, B.CP_SHARD_CONTIGUOUS),
+    (513, 128, 8, 2, B.CP_PASS_KV, B.CP_SHARD_LOAD_BALANCED),
+    (300, 1, 1, 1, B.CP_PASS_KV, B.CP_SHARD_LOAD_BALANCED),
+])
+def test_bf16_ring(t, n_h, n_kv, n_ranks, variant, mode):
+    pr = synth.make_prefill(t, n_h, n_kv, 128, "bf16", 100 + t, 0.5)
+    _run_prefill(pr, n_ranks, variant, mode)
+
+
+@pytest.mark.parametrize("q_scale", [1.0, 8.0])
+def test_bf16_persistent_kv_pass_q(q_scale):
+    """T new tokens over P cached + T keys, queries sharded and LSE-merged;
+    q_scale 8 makes the softmax peaked (|O| ~ |v|)."""
+    pr = synth.make_prefill(300, 32, 2, 128, "bf16", 7, 0.5, p=1500)
+    _run_prefill(pr, 4, B.CP_PASS_Q, B.CP_SHARD_LOAD_BALANCED, q_scale=q_scale)
+
+
+def test_bf16_varlen_running_merge():
+    lens = [700, 129, 1000]
+    segs, r0 = [], 0
+    for i, n in enumerate(lens):
+        segs.append(ring.Segment(n, r0, 0, i))
+        r0 += n
+    pr = synth.make_prefill(sum(lens), 16, 2, 128, "bf16", 5, 0.5)
+    _run_prefill(pr, 3, B.CP_PASS_KV, B.CP_SHARD_LOAD_BALANCED, merge="running", segs=segs)
+
+
+def test_bf16_partial_empty_rows():
+    rng = np.random.default_rng(4)
+    n_h, n_kv, d = 16, 1, 128
+    pr_q = synth.bf16_bits(rng.standard_normal((200, n_h, d)).astype(np.float32) * 0.5)
+    pr_k = synth.bf16_bits(rng.standard_normal((600, n_kv, d)).astype(np.float32) * 0.5)
+    pr_v = synth.bf16_bits(rng.standard_normal((600, n_kv, d)).astype(np.float32) * 0.5)
+    ranges = (B.cp_range * 2)(B.cp_range(3, 1000, 190, 0, 0), B.cp_range(7, 1050, 500, 0, 0))
+    blocks = (B.cp_block * 1)(B.cp_block(0, 1, 1, 1, 5))
+    o = torch.full((200, n_h, d), float("nan"), device="cuda")
+    lse = torch.full((200, n_h), float("nan"), device="cuda")
+    B.cp_attn_partial(dev(pr_q, "bf16"), dev(pr_k, "bf16"), dev(pr_v, "bf16"), n_h, n_kv, 1 / math.sqrt(d), True,
+                      ranges, 2, blocks, 1, o, lse, _ws())
+    torch.cuda.synchronize()
+    qv, kv, vv = (synth.bf16_bits_to_f32(x) for x in (pr_q, pr_k, pr_v))
+    o_ref, l_ref = OA.attention(qv[3:193], kv[7:507], vv[7:507], np.arange(1000, 1190), np.arange(1050, 1550))
+    check(o.cpu().numpy()[8:198], lse.cpu().numpy()[8:198], o_ref, l_ref, "bf16", "partial")
+    assert np.isnan(o.cpu().numpy()[:8]).all() and np.isnan(o.cpu().numpy()[198:]).all()   # untouched rows
+
+
+# ---------------------------------------------------------------------------- merge
+@pytest.mark.parametrize("n_parts,d,out_dtype", [(1, 128, "f32"), (3, 64, "f32"), (8, 128, "bf16"),
+                                                 (40, 128, "f32"), (256, 128, "bf16")])
+def test_merge(n_parts, d, out_dtype):
+    rng = np.random.default_rng(n_parts)
+    rows, n_h = 37, 4
+    o = rng.standard_normal((n_parts, rows, n_h, d)).astype(np.float32)
+    lse = (rng.standard_normal((n_parts, rows, n_h)) * 3).astype(np.float32)
+    lse[rng.random(lse.shape) < 0.2] = -np.inf
+    lse[:, 5, 1] = -np.inf      # a row-head with no part
+    o[np.isinf(lse)] = 0.0
+    o_ref, l_ref = OA.merge(list(o), list(lse))
+    out = torch.empty((rows, n_h, d), dtype=torch.bfloat16 if out_dtype == "bf16" else torch.float32, device="cuda")
+    lse_out = torch.empty((rows, n_h), dtype=torch.float32, device="cuda")
+    B.cp_attn_merge(dev(o, "f32"), dev(lse, "f32"), n_parts, rows, rows, n_h, d, out, lse_out)
+    torch.cuda.synchronize()
+    check(out.float().cpu().numpy(), lse_out.cpu().numpy(), o_ref, l_ref, "bf16" if out_dtype == "bf16" else "f32")
+
+
+def test_merge_in_place():
+    rng = np.random.default_rng(9)
+    rows, n_h, d = 64, 8, 128
+    o = rng.standard_normal((2, rows, n_h, d)).astype(np.float32)
+    lse = rng.standard_normal((2, rows, n_h)).astype(np.float32)
+    o_ref, l_ref = OA.merge(list(o), list(lse))
+    od, ld = dev(o, "f32"), dev(lse, "f32")
+    B.cp_attn_merge(od, ld, 2, rows, rows, n_h, d, od, ld)
+    torch.cuda.synchronize()
+    check(od[0].cpu().numpy(), ld[0].cpu().numpy(), o_ref, l_ref, "f32")
+
+
+# ---------------------------------------------------------------------------- decode
+@pytest.mark.parametrize("n_h,n_kv,n_splits", [(16, 1, 256), (16, 2, 16), (16, 1, 1), (64, 4, 256)])
+def test_decode(n_h, n_kv, n_splits):
+    lens = [0, 5, 100, 255, 256, 1000, 3001, 64]
+    dc = synth.make_decode(len(lens), n_h, n_kv, 128, lens, 40 + n_splits, 0.5)
+    q, k, v = dev(dc.q_raw, "bf16"), dev(dc.k_raw, "bf16"), dev(dc.v_raw, "bf16")
+    off = torch.from_numpy(dc.offsets).cuda()
+    out = torch.empty((len(lens), n_h, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((len(lens), n_h), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(B.cp_workspace_size(B.CP_OP_DECODE, len(lens), n_h, 128, n_splits), dtype=torch.uint8,
+                     device="cuda")
+    B.cp_decode(q, k, v, off, n_h, n_kv, n_splits, 1 / math.sqrt(128), out, lse, ws)
+    B.cp_check_status(ws)
+    o_ref, l_ref = OD.decode(dc.q, dc.k, dc.v, dc.offsets)
+    check(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "bf16", "decode")

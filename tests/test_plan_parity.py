@@ -1,0 +1,130 @@
+"""The C planner against the independent reference planner, bit for bit."""
+import itertools
+
+import numpy as np
+import pytest
+
+from context_ring_attn_b200 import binding as B
+from context_ring_attn_b200 import build as BUILD
+from context_ring_attn_b200 import synth
+from oracle import comm as OC
+from oracle import plan as OP
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    BUILD.build()
+    B.lib()
+
+
+def _segs(lens, pos0=None, seqs=None, row_base=0):
+    out, row = [], row_base
+    for i, ln in enumerate(lens):
+        out.append(OP.Segment(ln, row, 0 if pos0 is None else pos0[i], i if seqs is None else seqs[i]))
+        row += ln
+    return out
+
+
+def _c_segs(segs):
+    return B.segments([(s.length, s.row0, s.pos0, s.seq) for s in segs])
+
+
+def _ranges_equal(c_list, o_list):
+    assert len(c_list) == len(o_list)
+    for c, o in zip(c_list, o_list):
+        assert (c.row0, c.pos0, c.len, c.seq) == (o.row0, o.pos0, o.length, o.seq)
+
+
+CASES = [
+    ([256], 4), ([131072], 8), ([7], 4), ([1], 3), ([100, 37, 2], 3), ([5, 0, 9], 2),
+    (synth.varlen_lengths(1005), 8), ([126976], 8), ([4096], 8), ([1000], 1),
+]
+
+
+@pytest.mark.parametrize("lens,n", CASES)
+@pytest.mark.parametrize("mode", [OP.LOAD_BALANCED, OP.CONTIGUOUS])
+def test_shard_plan_bit_exact(lens, n, mode):
+    segs = _segs(lens)
+    cb, rr, ti = B.cp_shard_plan(_c_segs(segs), len(segs), n, mode)
+    ob, orr, oti = OP.shard_plan(segs, n, mode)
+    assert np.array_equal(cb, np.array(ob, dtype=np.int64).reshape(len(segs), 2 * n + 1))
+    assert list(rr) == orr
+    if len(oti) < 2_000_000:
+        assert np.array_equal(ti, np.array(oti, dtype=np.int64))
+    for r in range(n):
+        _ranges_equal(B.cp_rank_ranges(_c_segs(segs), len(segs), n, mode, r), OP.rank_ranges(segs, n, mode, r))
+
+
+def _schedule_case(kind):
+    if kind == "tiny":
+        s = _segs([256])
+        return s, s, 4
+    if kind == "prefill_128k":
+        s = _segs([131072])
+        return s, s, 8
+    if kind == "persistent_kv":
+        p, t = 126976, 4096
+        return [OP.Segment(t, 0, p, 0)], [OP.Segment(p, 0, 0, 0), OP.Segment(t, p, p, 0)], 8
+    if kind == "varlen":
+        s = _segs(synth.varlen_lengths(1005))
+        return s, s, 8
+    if kind == "ragged":
+        s = _segs([37, 5, 64], seqs=[0, 1, 2])
+        return s, s, 3
+
+
+@pytest.mark.parametrize("kind", ["tiny", "prefill_128k", "persistent_kv", "varlen", "ragged"])
+@pytest.mark.parametrize("mode", [OP.LOAD_BALANCED, OP.CONTIGUOUS])
+@pytest.mark.parametrize("variant", [OP.PASS_KV, OP.PASS_Q])
+def test_ring_schedule_bit_exact(kind, mode, variant):
+    q_segs, kv_segs, n = _schedule_case(kind)
+    ranges, n_ranges, blocks, parts = B.cp_ring_schedule(_c_segs(q_segs), len(q_segs), _c_segs(kv_segs),
+                                                         len(kv_segs), n, mode, variant)
+    o_ranges, o_blocks, o_parts = OP.ring_schedule(q_segs, kv_segs, n, mode, variant)
+    _ranges_equal([ranges[i] for i in range(n_ranges)], o_ranges)
+    assert parts == o_parts
+    for i, ob in enumerate(o_blocks):
+        cb = blocks[i]
+        assert (cb.q_begin, cb.q_count, cb.kv_begin, cb.kv_count, cb.out_row0) == \
+            (ob.q_begin, ob.q_count, ob.kv_begin, ob.kv_count, ob.out_row0)
+    # mask classes of every chunk pair, and the pair counts per block
+    for ob in o_blocks:
+        for a in range(ob.q_begin, ob.q_begin + ob.q_count):
+            for b in range(ob.kv_begin, ob.kv_begin + ob.kv_count):
+                assert B.cp_classify_pair(ranges[a], ranges[b], True) == OP.pair_class(o_ranges[a], o_ranges[b], True)
+                assert B.cp_classify_pair(ranges[a], ranges[b], False) == OP.pair_class(o_ranges[a], o_ranges[b], False)
+    if kind in ("tiny", "ragged"):
+        for i, ob in enumerate(o_blocks):
+            assert B.cp_block_pairs(ranges, blocks[i], True) == OP.block_pairs(o_ranges, ob, True)
+            assert B.cp_block_pairs(ranges, blocks[i], False) == OP.block_pairs(o_ranges, ob, False)
+    hops, total, a2a = B.cp_ring_comm_volume(ranges, blocks, n, variant, 128, 8, 128)
+    ref = OC.schedule_volume(o_ranges, o_blocks, n, variant, 128, 8, 128)
+    assert hops.tolist() == ref["hops"] and total == ref["total"] and a2a == ref["all_to_all"]
+
+
+def test_pair_counts_closed_form_prefill_128k():
+    """All blocks of the 128K schedule: C^2 + C(C+1) on the diagonal, 2C^2 elsewhere."""
+    n, c = 8, 8192
+    segs = _c_segs(_segs([2 * n * c]))
+    ranges, _, blocks, _ = B.cp_ring_schedule(segs, 1, segs, 1, n, B.CP_SHARD_LOAD_BALANCED, B.CP_PASS_KV)
+    total = 0
+    for t, i in itertools.product(range(n), range(n)):
+        want = c * c + c * (c + 1) if t == 0 else 2 * c * c
+        got = B.cp_block_pairs(ranges, blocks[t * n + i], True)
+        assert got == want
+        total += got
+    assert total == (2 * n * c) * (2 * n * c + 1) // 2
+
+
+def test_random_pairs_against_reference():
+    rng = np.random.default_rng(0)
+    for _ in range(500):
+        q = B.cp_range(0, int(rng.integers(0, 50)), int(rng.integers(0, 30)), int(rng.integers(0, 2)), 0)
+        k = B.cp_range(0, int(rng.integers(0, 50)), int(rng.integers(0, 30)), int(rng.integers(0, 2)), 0)
+        oq = OP.Range(0, q.pos0, q.len, q.seq)
+        ok = OP.Range(0, k.pos0, k.len, k.seq)
+        ranges = (B.cp_range * 2)(q, k)
+        blk = B.cp_block(0, 1, 1, 1, 0)
+        for causal in (True, False):
+            assert B.cp_classify_pair(q, k, causal) == OP.pair_class(oq, ok, causal)
+            assert B.cp_block_pairs(ranges, blk, causal) == OP.visible_pairs(oq, ok, causal)
