@@ -1,0 +1,468 @@
+"""Benchmark of the context-parallel ring-attention hot path on B200.
+
+One step = one pass of the hot path over the 128K full-prefill workload:
+the load-balanced shard plan for 8 virtual ranks (host), the 8 pass-KV ring
+steps (one cp_attn_partial launch each, tcgen05 kernel) and the 8-way LSE
+merge into the bf16 output. Workload: Llama3-405B per-TP8-rank head slice,
+N_H=16, N_KV=1, D_H=128, T=131072, bf16 inputs iid N(0,1)*0.5 (seeded,
+synthetic). The split-KV decode workload (32 requests, 256 splits) is timed
+in the same run and reported under "decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 (launched by torchrun): every rank runs its own copy of the workload
+(independent replicas, weak scaling, no data-path collective); the time is
+the max over ranks and `value` counts the work of all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "causal prefill attn TFLOP/s; decode KV GB/s; % of B200 roofline, 1 GPU"
+WORKLOAD = "prefill_128k"
+DECODE = "decode_split"
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "partial_bf16_prefill_128k.txt")
+KERNEL_SOURCES = ["context_ring_attn_b200/csrc/partial_tc.cuh", "context_ring_attn_b200/csrc/common.cuh",
+                  "context_ring_attn_b200/csrc/work.cuh"]
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def profiled_traffic():
+    """Per-launch DRAM bytes of the partial kernel from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    vals = {}
+    with open(PROFILE_TRAFFIC) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_hash") != kernel_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch_full_size"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------ reference arm
+def oracle_sample(budget_s: float, seed_tokens: int = 0):
+    """Time the fp64 oracle on sampled query tokens of the 128K prefill (all 16
+    heads, each token against its causal prefix). Returns (flops, seconds, n_tokens)."""
+    from context_ring_attn_b200 import synth
+    from oracle import attention as OA
+
+    w = synth.WORKLOADS[WORKLOAD]
+    t, n_h, n_kv, d = w["t"], w["n_h"], w["n_kv"], w["d"]
+    k = synth.stored_values(synth.normal_rows(w["seed"], synth.TENSOR_K, t, (n_kv, d), w["std"]), "bf16")[0]
+    v = synth.stored_values(synth.normal_rows(w["seed"], synth.TENSOR_V, t, (n_kv, d), w["std"]), "bf16")[0]
+    k64, v64 = k.astype(np.float64), v.astype(np.float64)
+    rng = np.random.default_rng(12345 + seed_tokens)
+    flops, spent, n_tok = 0.0, 0.0, 0
+    k_pos = np.arange(t)
+    while spent < budget_s or n_tok < 4:
+        tok = int(rng.integers(0, t))
+        qrow = synth.stored_values(synth.normal_rows(w["seed"], synth.TENSOR_Q, t, (n_h, d), w["std"], [tok]),
+                                   "bf16")[0]
+        t0 = time.perf_counter()
+        OA.attention(qrow, k64[:tok + 1], v64[:tok + 1], np.array([tok]), k_pos[:tok + 1])
+        spent += time.perf_counter() - t0
+        flops += 4.0 * d * n_h * (tok + 1)
+        n_tok += 1
+    return flops, spent, n_tok
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            return max(int(i.get("num_threads", 1)) for i in info)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return
+    cores = blas_threads()
+    per_step = max(2.0, min(8.0, 120.0 / max(1, args.steps)))
+    oracle_sample(0.5)  # warm caches and BLAS threads (not timed)
+    for _ in range(args.warmup):
+        oracle_sample(0.5)
+    flops = secs = 0.0
+    toks = 0
+    for _ in range(args.steps):
+        f, s, n = oracle_sample(per_step)
+        flops, secs, toks = flops + f, secs + s, toks + n
+    value = flops / secs / 1e12
+    sample = (f"{toks} query tokens of the 128K causal prefill drawn at random positions, all 16 heads, "
+              f"fp64 numpy, each against its whole causal prefix; {args.steps} steps of ~{per_step:.0f} s")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "T": 131072, "N_H": 16, "N_KV": 1, "D_H": 128, "cp_ranks": 8,
+                   "plan": "load-balanced 16 chunks", "ring": "pass-KV"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------ our arm
+def run_ours(args, rank: int, world: int):
+    import torch
+    import torch.distributed as dist
+
+    from context_ring_attn_b200 import binding as B
+    from context_ring_attn_b200 import ring, synth
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = synth.WORKLOADS[WORKLOAD]
+    t, n_h, n_kv, d, n_ranks = w["t"], w["n_h"], w["n_kv"], w["d"], w["n_ranks"]
+    if args.tokens:
+        t = args.tokens
+    scale = 1.0 / math.sqrt(d)
+    q = synth.device_rows(w["seed"], synth.TENSOR_Q, t, (n_h, d), w["std"], "bf16", dev)
+    k = synth.device_rows(w["seed"], synth.TENSOR_K, t, (n_kv, d), w["std"], "bf16", dev)
+    v = synth.device_rows(w["seed"], synth.TENSOR_V, t, (n_kv, d), w["std"], "bf16", dev)
+    segs = [ring.Segment(t, 0, 0, 0)]
+    o_parts, lse_parts = ring.partial_buffers(t, n_h, d, n_ranks, dev)
+    out = torch.empty((t, n_h, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((t, n_h), dtype=torch.float32, device=dev)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    sched0 = ring.RingSchedule(segs, segs, n_ranks, B.CP_PASS_KV)
+    pairs = sched0.pairs(True)
+    step_flops = 4.0 * d * n_h * pairs
+    step_pairs = [sum(B.cp_block_pairs(sched0.ranges, sched0.blocks[s * n_ranks + i], True)
+                      for i in range(n_ranks)) for s in range(n_ranks)]
+
+    ev_part = []  # (start, end, flops) of each partial launch in the timed region
+    ev_merge = []
+
+    def step(record: bool):
+        sched = ring.RingSchedule(segs, segs, n_ranks, B.CP_PASS_KV)   # host plan, every step
+        for s in range(n_ranks):
+            blocks = sched.step_blocks(s, t)
+            if record:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            B.cp_attn_partial(q, k, v, n_h, n_kv, scale, True, sched.ranges, sched.n_ranges, blocks, n_ranks,
+                              o_parts, lse_parts, ws)
+            if record:
+                e1.record(stream)
+                ev_part.append((e0, e1, 4.0 * d * n_h * step_pairs[s]))
+        if record:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        B.cp_attn_merge(o_parts, lse_parts, n_ranks, t, t, n_h, d, out, lse)
+        if record:
+            e1.record(stream)
+            ev_merge.append((e0, e1))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    B.cp_check_status(ws)
+
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step(True)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop() if clocks else None
+    B.cp_check_status(ws)
+    elapsed_ms = t_start.elapsed_time(t_end)
+    part_ms = sum(a.elapsed_time(b) for a, b, _ in ev_part)
+    part_flops = sum(f for _, _, f in ev_part)
+    merge_ms = sum(a.elapsed_time(b) for a, b in ev_merge)
+    if world > 1:
+        tt = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+
+    e2e = run_e2e(args, q, k, v, out, lse, o_parts, lse_parts, ws, segs, n_ranks, n_h, n_kv, world, dev,
+                  step_flops, barrier) if not args.no_e2e else None
+    decode = run_decode(args, dev) if not args.no_decode else None
+
+    if rank != 0:
+        return
+    peaks, peak_kind = load_peaks()
+    peak_t = float(peaks["bf16_tflops_sustained"])
+    achieved = part_flops / (part_ms * 1e-3) / 1e12
+    traffic = profiled_traffic() if t == w["t"] else None
+    value = world * step_flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+    merge_bytes = n_ranks * t * n_h * (d + 1) * 4 + t * n_h * (d * 2 + 4)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD if t == w["t"] else f"{WORKLOAD} (T={t} profiling variant)",
+                   "T": t, "N_H": n_h, "N_KV": n_kv, "D_H": d, "cp_ranks": n_ranks,
+                   "plan": "load-balanced 16 chunks", "ring": "pass-KV", "merge": "final 8-way",
+                   "flops_per_step": step_flops, "causal_pairs_per_head": pairs,
+                   "l2": "no flush: inputs larger than L2 (Q 537 MB, partials 8.6 GB per step)",
+                   "parallelism": f"{world} independent replica(s)"},
+        "roofline": {"kernel": "partial_bf16_kernel", "bound": "tensor", "achieved": achieved, "peak": peak_t,
+                     "unit": "TFLOP/s", "frac": achieved / peak_t, "traffic": traffic,
+                     "peak_kind": f"bf16_tflops_sustained ({peak_kind})",
+                     "kernel_ms_per_step": part_ms / args.steps},
+        "merge": {"ms_per_step": merge_ms / args.steps,
+                  "gbs": merge_bytes / (merge_ms / args.steps * 1e-3) / 1e9,
+                  "frac_hbm": merge_bytes / (merge_ms / args.steps * 1e-3) / 1e9 / float(peaks["hbm_gbs"])},
+        "e2e": e2e,
+        "gpu_launches": args.steps * (n_ranks + 1),
+        "clocks": clk,
+    }
+    if decode:
+        line["decode"] = decode
+    if not args.no_cpu_baseline:
+        f, s, n = oracle_sample(args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": f / s / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} query tokens of the 128K causal prefill at random positions, all 16 heads, fp64 numpy "
+                      f"against each token's causal prefix ({s:.1f} s)"}
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, q, k, v, out, lse, o_parts, lse_parts, ws, segs, n_ranks, n_h, n_kv, world, dev, step_flops,
+            barrier):
+    import torch
+    import torch.distributed as dist
+
+    from context_ring_attn_b200 import binding as B
+    from context_ring_attn_b200 import ring
+
+    stream = torch.cuda.current_stream()
+    # ---- end to end through the public API with host buffers (pinned), per step:
+    # H2D of Q, K, V; the ring; D2H of O and LSE.
+    q_h = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    k_h = torch.empty(k.shape, dtype=k.dtype, pin_memory=True)
+    v_h = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+    o_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    l_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    q_h.copy_(q)
+    k_h.copy_(k)
+    v_h.copy_(v)
+    torch.cuda.synchronize()
+
+    def e2e_step():
+        q.copy_(q_h, non_blocking=True)
+        k.copy_(k_h, non_blocking=True)
+        v.copy_(v_h, non_blocking=True)
+        ring.run_ring(ring.RingSchedule(segs, segs, n_ranks, B.CP_PASS_KV), q, k, v, n_h, n_kv, out, lse,
+                      o_parts=o_parts, lse_parts=lse_parts, workspace=ws)
+        o_h.copy_(out, non_blocking=True)
+        l_h.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(2, args.steps // 2)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    h2d = (q.numel() + k.numel() + v.numel()) * 2
+    d2h = out.numel() * 2 + lse.numel() * 4
+    del q_h, k_h, v_h, o_h, l_h
+    return {"value": world * step_flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def run_decode(args, dev):
+    """Split-KV decode: 32 requests, 16 heads on 1 KV head, 256 splits; GB/s
+    of K/V read (each byte once)."""
+    import torch
+
+    from context_ring_attn_b200 import binding as B
+    from context_ring_attn_b200 import synth
+
+    w = synth.WORKLOADS[DECODE]
+    lens = synth.decode_lengths(w["seed"], w["batch"], w["lo"], w["hi"])
+    offsets = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    total = int(offsets[-1])
+    b, n_h, n_kv, d, ns = w["batch"], w["n_h"], w["n_kv"], w["d"], w["n_splits"]
+    q = synth.device_rows(w["seed"], synth.TENSOR_Q, b, (n_h, d), w["std"], "bf16", dev)
+    k = synth.device_rows(w["seed"], synth.TENSOR_K, total, (n_kv, d), w["std"], "bf16", dev)
+    v = synth.device_rows(w["seed"], synth.TENSOR_V, total, (n_kv, d), w["std"], "bf16", dev)
+    off = torch.from_numpy(offsets).to(dev)
+    out = torch.empty((b, n_h, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((b, n_h), dtype=torch.float32, device=dev)
+    ws = torch.zeros(B.cp_workspace_size(B.CP_OP_DECODE, b, n_h, d, ns), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        B.cp_decode(q, k, v, off, n_h, n_kv, ns, 1 / math.sqrt(d), out, lse, ws)
+    torch.cuda.synchronize()
+    times = []
+    iters = max(10, args.steps)
+    for _ in range(iters):
+        flush.fill_(1)            # evict K/V from L2 between iterations
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        B.cp_decode(q, k, v, off, n_h, n_kv, ns, 1 / math.sqrt(d), out, lse, ws)
+        e1.record(stream)
+        times.append((e0, e1))
+    torch.cuda.synchronize()
+    B.cp_check_status(ws)
+    ms = statistics.median(a.elapsed_time(c) for a, c in times)
+    kv_bytes = total * n_kv * d * 2 * 2
+    peaks, kind = load_peaks()
+    gbs = kv_bytes / (ms * 1e-3) / 1e9
+    return {"value": gbs, "unit": "GB/s", "ms": ms, "kv_bytes": kv_bytes, "batch": b, "n_splits": ns,
+            "frac_hbm": gbs / float(peaks["hbm_gbs"]), "peak": float(peaks["hbm_gbs"]),
+            "peak_kind": f"hbm_gbs ({kind})", "l2": "256 MB buffer written between iterations",
+            "note": "split kernel + 256-way merge, median of iterations"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only-decode", action="store_true", help="time the split-KV decode workload alone")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="shorter sequence for profiling captures (default: the full 131072)")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import torch
+    import torch.distributed as dist
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    try:
+        if args.only_decode:
+            print(json.dumps({"decode": run_decode(args, torch.device("cuda", local))}), flush=True)
+            return
+        run_ours(args, rank, world)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
