@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libcpattn.so")
 SOURCES = ["plan.cpp", "capi.cu"]
-HEADERS = ["common.cuh", "work.cuh", "partial_tc.cuh", "partial_simt.cuh", "merge.cuh", "decode.cuh"]
+HEADERS = ["common.cuh", "work.cuh", "partial_tc.cuh", "partial_simt.cuh", "merge.cuh", "decode.cuh", "exp2_poly.cuh"]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",

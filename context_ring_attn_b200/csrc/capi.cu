@@ -264,7 +264,8 @@ cp_status cp_attn_partial(const void* q, const void* k, const void* v, cp_dtype 
       if (!range_ok(r) || r.row0 + r.len > kv_rows) return CP_ERR_INVALID_ARG;
     }
   }
-  const int tok_per_tile = (dtype == CP_BF16) ? 128 / group : simt::kRows / group;
+  // tokens per CTA tile: the tensor-core kernel takes two 128-row query tiles per CTA
+  const int tok_per_tile = (dtype == CP_BF16) ? tc::kQTiles * (128 / group) : simt::kRows / group;
   std::vector<WorkTable> tables;
   if (!build_tables(ranges, blocks, n_blocks, tok_per_tile, causal != 0, tables)) return CP_ERR_UNSUPPORTED;
 

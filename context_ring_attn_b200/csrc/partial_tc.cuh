@@ -8,18 +8,24 @@
 // exact attention, "Context Parallelism과 Expert Parallelism" section 4.1), so
 // the block yields O normalised within the block plus its log-sum-exp.
 //
-// One CTA = one 128-row query tile of one KV head. GQA packing: the 128 rows
-// are (token, head-in-group) pairs, 128/G tokens x G query heads that share
-// the KV head (section 8.2 of the GQA page), so every K/V tile is loaded once
-// for all G heads. Warp roles (192 threads):
-//   warps 0-3  softmax: thread = query row; reads S rows from TMEM, masks by
-//              global position, online max/sum, writes P (bf16) to shared
-//              memory, rescales O in TMEM when the running max moves by more
-//              than 2^8, and writes the normalised O and LSE at the end;
-//   warp 4     TMA producer: Q once, then K and V tiles into a 2-stage ring;
-//   warp 5     MMA issuer (one thread): S = Q K^T into a double-buffered TMEM
-//              slot, O += P V into the TMEM accumulator; owns TMEM alloc.
-// TMEM (512 columns): S buffers at columns 0 and 128, O at 256.
+// One CTA = two 128-row query tiles (a, b) of one KV head. GQA packing: each
+// tile's rows are (token, head-in-group) pairs, 128/G tokens x G query heads
+// that share the KV head (section 8.2 of the GQA page), so every K/V tile is
+// loaded once for 2 x 128 rows. Warp roles (320 threads):
+//   warps 0-3  softmax of tile a, warps 4-7 softmax of tile b: thread = row.
+//              It reads its S row from TMEM, masks by global position, keeps
+//              the running max, writes P (bf16 pairs) over its own S row in
+//              TMEM, rescales its O row in TMEM when the running max grows by
+//              more than 2^8, and writes the normalised O row and its LSE;
+//   warp 8     TMA producers: lane 0 loads Q, then K tiles into a 3-stage
+//              ring; lane 1 loads V tiles into a 2-stage ring;
+//   warp 9     MMA issuer (one thread) and TMEM owner. Per KV tile j it issues
+//              O_a += P_a(j) V_j, S_a(j+1) = Q_a K_{j+1}^T, O_b += P_b(j) V_j,
+//              S_b(j+1) = Q_b K_{j+1}^T, so that one tile's softmax always
+//              overlaps the other tile's MMAs (ping-pong).
+// TMEM (512 columns): S_a 0, S_b 128 (P over the first 64 columns), O_a 256,
+// O_b 384. tcgen05 operations of one thread complete in issue order, so the
+// completion of S_x(j+1) also means O_x += P_x(j) V_j has completed.
 #pragma once
 
 #include "common.cuh"
@@ -31,35 +37,44 @@ namespace tc {
 constexpr int BM = 128;                      // packed query rows per tile
 constexpr int BN = 128;                      // keys per KV tile
 constexpr int HD = 128;                      // head dim
+constexpr int kQTiles = 2;                   // query tiles per CTA
 constexpr int kHalfBytes = 128 * 128;        // 128 rows x 64 bf16 (one 128-byte swizzle column)
 constexpr int kTileBytes = 2 * kHalfBytes;   // 128 rows x 128 bf16
-constexpr int kStages = 2;
-constexpr int kThreads = 192;
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kTileBytes;
-constexpr int kOffV = kOffK + kStages * kTileBytes;
-constexpr int kOffP = kOffV + kStages * kTileBytes;
-constexpr int kOffBar = kOffP + kTileBytes;
-constexpr int kNumBars = 16;
+constexpr int kOffK = kOffQ + kQTiles * kTileBytes;
+constexpr int kOffV = kOffK + kKStages * kTileBytes;
+constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+constexpr int kNumBars = 24;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + slack to align the base to 1024
+constexpr int kSmemNeeded = kOffMisc + 16;
+constexpr int kSmemMax = 232448;                     // 227 KB per block on sm_100
+// The dynamic shared window starts 1024-aligned in practice; whatever slack is
+// left covers a smaller alignment, and the kernel checks it at run time.
+constexpr int kSmemBytes = kSmemNeeded + 1024 <= kSmemMax ? kSmemNeeded + 1024 : kSmemMax;
+static_assert(kSmemNeeded <= kSmemMax, "shared memory plan exceeds 227 KB");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;
-constexpr uint32_t kColO = 256;
+constexpr uint32_t kColS = 0;     // + tile * 128
+constexpr uint32_t kColO = 256;   // + tile * 128
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled when the max grows by > 2^8
+constexpr int kPolyPairsPer8 = 2;          // of every 8 column pairs, this many take the polynomial exp2
 
 // barrier slots
 enum {
   B_Q_FULL = 0,
-  B_K_FULL = 1,   // +stage
-  B_V_FULL = 3,   // +stage
-  B_K_EMPTY = 5,  // +stage
-  B_V_EMPTY = 7,  // +stage
-  B_S_FULL = 9,   // +buffer
-  B_S_FREE = 11,  // +buffer
-  B_P_FULL = 13,
-  B_PV_DONE = 14,
-  B_DRAIN = 15
+  B_K_FULL = 1,     // +stage (3)
+  B_K_EMPTY = 4,    // +stage (3)
+  B_V_FULL = 7,     // +stage (2)
+  B_V_EMPTY = 9,    // +stage (2)
+  B_S_FULL = 11,    // +tile: S_x(j) is in TMEM (and O_x += P_x(j-1) V is done)
+  B_P_FULL = 13,    // +tile (4 arrivals): P_x(j) is in TMEM
+  B_O_DONE = 15,    // +tile: O_x += P_x(j) V_j has completed
+  B_DRAIN = 17
 };
 
 struct Params {
@@ -73,7 +88,7 @@ struct Params {
   int32_t log2_group;
   int32_t causal;
   float scale_log2;  // softmax scale * log2(e)
-  WorkTable wt;
+  WorkTable wt;      // tiles here are 256-row CTA tiles (two query tiles)
 };
 
 // Wait on a barrier with every lane of the warp; the outcome is made
@@ -105,6 +120,10 @@ __global__ void __launch_bounds__(kThreads, 1) partial_bf16_kernel(const __grid_
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  if (pad + kSmemNeeded > kSmemBytes) {  // uniform across the CTA: nothing has started yet
+    if (threadIdx.x == 0) atomicOr(p.status, kStatusInternal);
+    return;
+  }
 
   int32_t seg, tile;
   locate_tile(p.wt, blockIdx.x, seg, tile);
@@ -112,15 +131,15 @@ __global__ void __launch_bounds__(kThreads, 1) partial_bf16_kernel(const __grid_
   const cp_range qr = p.wt.ranges[ws.q_range];
   const int kvh = blockIdx.y;
   const int group = 1 << p.log2_group;
-  const int tok_per_tile = BM >> p.log2_group;
-  const int64_t tok0 = static_cast<int64_t>(tile) * tok_per_tile;
-  const int n_tok = static_cast<int>(min(static_cast<int64_t>(tok_per_tile), qr.len - tok0));
+  const int tok_per_tile = BM >> p.log2_group;            // tokens per 128-row query tile
+  const int64_t tok0 = static_cast<int64_t>(tile) * (kQTiles * tok_per_tile);
+  const int n_tok = static_cast<int>(min(static_cast<int64_t>(kQTiles * tok_per_tile), qr.len - tok0));
   const int64_t q_row0 = qr.row0 + tok0;
   const int64_t q_pos_lo = qr.pos0 + tok0;
   const int64_t q_pos_hi = q_pos_lo + n_tok - 1;
   const int causal = p.causal;
 
-  // number of KV tiles this query tile visits
+  // KV tiles the CTA visits (enough for its last valid token)
   int n_iter = 0;
   for (int r = 0; r < ws.kv_count; ++r) {
     const cp_range kr = p.wt.ranges[ws.kv_begin + r];
@@ -129,19 +148,15 @@ __global__ void __launch_bounds__(kThreads, 1) partial_bf16_kernel(const __grid_
   }
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNumBars; ++i) {
-      uint32_t count = 1;
-      if (i == B_S_FREE || i == B_S_FREE + 1 || i == B_P_FULL) count = 4;  // one arrive per softmax warp
-      mbar_init(&bars[i], count);
-    }
+    for (int i = 0; i < kNumBars; ++i) mbar_init(&bars[i], (i == B_P_FULL || i == B_P_FULL + 1) ? 4u : 1u);
     *abort_flag = 0u;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     prefetch_tensormap(&p.tm_q);
     prefetch_tensormap(&p.tm_k);
     prefetch_tensormap(&p.tm_v);
@@ -154,16 +169,25 @@ __global__ void __launch_bounds__(kThreads, 1) partial_bf16_kernel(const __grid_
   uint8_t* sQ = smem + kOffQ;
   uint8_t* sK = smem + kOffK;
   uint8_t* sV = smem + kOffV;
-  uint8_t* sP = smem + kOffP;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0 && n_iter > 0) {
-      uint32_t issued_k[kStages] = {0u, 0u};
-      uint32_t issued_v[kStages] = {0u, 0u};
-      mbar_arrive_expect_tx(&bars[B_Q_FULL], kTileBytes);
-      tma_load_4d(sQ, &p.tm_q, &bars[B_Q_FULL], 0, 0, kvh, static_cast<int>(q_row0));
-      tma_load_4d(sQ + kHalfBytes, &p.tm_q, &bars[B_Q_FULL], 64, 0, kvh, static_cast<int>(q_row0));
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------------ TMA producers
+    if (lane < 2 && n_iter > 0) {
+      const bool is_k = lane == 0;
+      const int n_st = is_k ? kKStages : kVStages;
+      uint8_t* base = is_k ? sK : sV;
+      const CUtensorMap* map = is_k ? &p.tm_k : &p.tm_v;
+      uint64_t* full = &bars[is_k ? B_K_FULL : B_V_FULL];
+      uint64_t* empty = &bars[is_k ? B_K_EMPTY : B_V_EMPTY];
+      uint32_t issued[kKStages] = {0u, 0u, 0u};
+      if (is_k) {
+        mbar_arrive_expect_tx(&bars[B_Q_FULL], kQTiles * kTileBytes);
+        for (int t = 0; t < kQTiles; ++t) {
+          const int row = static_cast<int>(q_row0) + t * tok_per_tile;
+          tma_load_4d(sQ + t * kTileBytes, &p.tm_q, &bars[B_Q_FULL], 0, 0, kvh, row);
+          tma_load_4d(sQ + t * kTileBytes + kHalfBytes, &p.tm_q, &bars[B_Q_FULL], 64, 0, kvh, row);
+        }
+      }
       int it = 0;
       bool ok = true;
       for (int r = 0; r < ws.kv_count && ok; ++r) {
@@ -171,81 +195,83 @@ __global__ void __launch_bounds__(kThreads, 1) partial_bf16_kernel(const __grid_
         if (kr.seq != qr.seq) continue;
         const int64_t nv = visible_keys(kr, q_pos_hi, causal);
         for (int64_t k0 = 0; k0 < nv; k0 += BN, ++it) {
-          const int st = it & 1;
-          const uint32_t ph = (it >> 1) & 1;
+          const int st = it % n_st;
+          const uint32_t ph = (it / n_st) & 1;
           const int key_row = static_cast<int>(kr.row0 + k0);
-          if (it >= 2 && !mbar_wait(&bars[B_K_EMPTY + st], ph ^ 1u, abort_flag, p.status)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars[B_K_FULL + st], kTileBytes);
-          tma_load_3d(sK + st * kTileBytes, &p.tm_k, &bars[B_K_FULL + st], 0, kvh, key_row);
-          tma_load_3d(sK + st * kTileBytes + kHalfBytes, &p.tm_k, &bars[B_K_FULL + st], 64, kvh, key_row);
-          issued_k[st] += 1;
-          if (it >= 2 && !mbar_wait(&bars[B_V_EMPTY + st], ph ^ 1u, abort_flag, p.status)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars[B_V_FULL + st], kTileBytes);
-          tma_load_3d(sV + st * kTileBytes, &p.tm_v, &bars[B_V_FULL + st], 0, kvh, key_row);
-          tma_load_3d(sV + st * kTileBytes + kHalfBytes, &p.tm_v, &bars[B_V_FULL + st], 64, kvh, key_row);
-          issued_v[st] += 1;
+          if (it >= n_st && !mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[st], kTileBytes);
+          tma_load_3d(base + st * kTileBytes, map, &full[st], 0, kvh, key_row);
+          tma_load_3d(base + st * kTileBytes + kHalfBytes, map, &full[st], 64, kvh, key_row);
+          issued[st] += 1;
         }
       }
       // Drain: every load issued has landed before the CTA may exit.
-      drain_wait(&bars[B_Q_FULL], 0u, p.status);
-      for (int st = 0; st < kStages; ++st) {
-        if (issued_k[st] > 0) drain_wait(&bars[B_K_FULL + st], (issued_k[st] - 1u) & 1u, p.status);
-        if (issued_v[st] > 0) drain_wait(&bars[B_V_FULL + st], (issued_v[st] - 1u) & 1u, p.status);
-      }
+      if (is_k) drain_wait(&bars[B_Q_FULL], 0u, p.status);
+      for (int st = 0; st < n_st; ++st)
+        if (issued[st] > 0) drain_wait(&full[st], (issued[st] - 1u) & 1u, p.status);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_iter > 0) {
       constexpr uint32_t idesc_s = umma_idesc_bf16(BM, BN, 0);   // Q, K both K-major
-      constexpr uint32_t idesc_o = umma_idesc_bf16(BM, HD, 1);   // P K-major, V MN-major
+      constexpr uint32_t idesc_o = umma_idesc_bf16(BM, HD, 1);   // P (TMEM) K-major, V MN-major
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t k_addr = smem_u32(sK);
       const uint32_t v_addr = smem_u32(sV);
-      const uint32_t p_addr = smem_u32(sP);
-      auto issue_pv = [&](int j) -> bool {
-        if (!mbar_wait(&bars[B_P_FULL], j & 1, abort_flag, p.status)) return false;
-        if (!mbar_wait(&bars[B_V_FULL + (j & 1)], (j >> 1) & 1, abort_flag, p.status)) return false;
-        tc_fence_after();
-        const uint32_t vb = v_addr + (j & 1) * kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint64_t a = umma_sdesc_sw128(p_addr + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = umma_sdesc_sw128(vb + kk * 2048, kHalfBytes, 1024);
-          umma_bf16_ss(tmem + kColO, a, b, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&bars[B_PV_DONE]);
-        umma_commit(&bars[B_V_EMPTY + (j & 1)]);
-        return true;
-      };
-      bool ok = mbar_wait(&bars[B_Q_FULL], 0u, abort_flag, p.status);
-      for (int it = 0; it < n_iter && ok; ++it) {
-        const int st = it & 1;
-        const uint32_t ph = (it >> 1) & 1;
-        if (!mbar_wait(&bars[B_K_FULL + st], ph, abort_flag, p.status)) { ok = false; break; }
-        if (it >= 2 && !mbar_wait(&bars[B_S_FREE + st], ph ^ 1u, abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t kb = k_addr + st * kTileBytes;
+      auto issue_s = [&](int x, int i) {   // S_x(i) = Q_x K_i^T
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          const uint64_t a = umma_sdesc_sw128(q_addr + off, 16, 1024);
-          const uint64_t b = umma_sdesc_sw128(kb + off, 16, 1024);
-          umma_bf16_ss(tmem + kColS + st * BN, a, b, idesc_s, kk > 0 ? 1u : 0u);
+          const uint64_t a = umma_sdesc_sw128(q_addr + x * kTileBytes + off, 16, 1024);
+          const uint64_t b = umma_sdesc_sw128(k_addr + (i % kKStages) * kTileBytes + off, 16, 1024);
+          umma_bf16_ss(tmem + kColS + x * BN, a, b, idesc_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bars[B_S_FULL + st]);
-        umma_commit(&bars[B_K_EMPTY + st]);
-        if (it >= 1 && !issue_pv(it - 1)) { ok = false; break; }
+        umma_commit(&bars[B_S_FULL + x]);
+      };
+      auto issue_pv = [&](int x, int j) {  // O_x += P_x(j) V_j
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t b = umma_sdesc_sw128(v_addr + (j % kVStages) * kTileBytes + kk * 2048, kHalfBytes, 1024);
+          umma_bf16_ts(tmem + kColO + x * HD, tmem + kColS + x * BN + kk * 8, b, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&bars[B_O_DONE + x]);
+      };
+      bool ok = mbar_wait(&bars[B_Q_FULL], 0u, abort_flag, p.status) &&
+                mbar_wait(&bars[B_K_FULL], 0u, abort_flag, p.status);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        umma_commit(&bars[B_K_EMPTY]);
       }
-      if (ok) issue_pv(n_iter - 1);
+      for (int j = 0; j < n_iter && ok; ++j) {
+        const bool more = j + 1 < n_iter;
+        const int kn = (j + 1) % kKStages;
+        if (!mbar_wait(&bars[B_V_FULL + j % kVStages], (j / kVStages) & 1, abort_flag, p.status)) { ok = false; break; }
+        if (more && !mbar_wait(&bars[B_K_FULL + kn], ((j + 1) / kKStages) & 1, abort_flag, p.status)) { ok = false; break; }
+        for (int x = 0; x < kQTiles; ++x) {
+          if (!mbar_wait(&bars[B_P_FULL + x], j & 1, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(x, j);
+          if (more) issue_s(x, j + 1);
+        }
+        if (!ok) break;
+        umma_commit(&bars[B_V_EMPTY + j % kVStages]);
+        if (more) umma_commit(&bars[B_K_EMPTY + kn]);
+      }
       // Everything this thread issued completes before TMEM is released.
       umma_commit(&bars[B_DRAIN]);
       drain_wait(&bars[B_DRAIN], 0u, p.status);
     }
   } else {
-    // ------------------------------------------------------------------ softmax warps 0..3
-    const int row = threadIdx.x;  // TMEM lane == packed query row
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const int tok = row >> p.log2_group;
+    // ------------------------------------------------------------------ softmax warps 0..7
+    const int x = warp >> 2;                // query tile of this warpgroup
+    const int quarter = warp & 3;           // TMEM lane quarter
+    const int row = quarter * 32 + lane;    // packed row within the tile
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t s_col = tmem + lane_base + kColS + x * BN;
+    const uint32_t o_col = tmem + lane_base + kColO + x * HD;
+    const int tok = x * tok_per_tile + (row >> p.log2_group);   // token within the CTA
     const bool row_valid = tok < n_tok;
     const int64_t qpos = q_pos_lo + tok;
     const float sl2 = p.scale_log2;
@@ -259,35 +285,42 @@ __global__ void __launch_bounds__(kThreads, 1) partial_bf16_kernel(const __grid_
       if (kr.seq != qr.seq) continue;
       const int64_t nv = visible_keys(kr, q_pos_hi, causal);
       for (int64_t k0 = 0; k0 < nv; k0 += BN, ++it) {
-        const int sb = it & 1;
         const int64_t kp0 = kr.pos0 + k0;
         const int n_valid = static_cast<int>(min(static_cast<int64_t>(BN), nv - k0));
-        const bool need_mask = (n_valid < BN) || (causal && kp0 + BN - 1 > q_pos_lo);
-
-        if (!warp_wait(&bars[B_S_FULL + sb], (it >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        // S_x(it) is in TMEM; this also means O_x += P_x(it-1) V has completed
+        if (!warp_wait(&bars[B_S_FULL + x], it & 1, abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
         uint32_t s[4][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + kColS + sb * BN + c * 32, s[c]);
+        for (int c = 0; c < 4; ++c) tmem_ld32(s_col + c * 32, s[c]);
         tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[B_S_FREE + sb]);
 
-        if (need_mask) {
-          // key c is visible iff c < n_valid and (not causal or kp0 + c <= qpos)
-          int64_t lim = n_valid - 1;
-          if (causal) {
-            const int64_t c_lim = qpos - kp0;
-            if (c_lim < lim) lim = c_lim;
-          }
+        // key c of the tile is visible iff c <= lim
+        int lim = BN - 1;
+        if ((n_valid < BN) || (causal && kp0 + BN - 1 > qpos)) {
+          int64_t l64 = n_valid - 1;
+          if (causal && qpos - kp0 < l64) l64 = qpos - kp0;
+          lim = static_cast<int>(max(l64, static_cast<int64_t>(-1)));
+        }
+        const bool masked = __any_sync(0xffffffffu, lim < BN - 1);
+        if (masked) {
 #pragma unroll
           for (int c = 0; c < BN; ++c)
             if (c > lim) s[c >> 5][c & 31] = __float_as_uint(-INFINITY);
         }
-        float mx = -INFINITY;
+        // row max: four chains of 3-input max
+        float mx;
+        {
+          float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, __uint_as_float(s[c >> 5][c & 31]));
+          for (int c = 0; c < BN; c += 8) {
+            a0 = fmax3(a0, __uint_as_float(s[c >> 5][(c + 0) & 31]), __uint_as_float(s[c >> 5][(c + 1) & 31]));
+            a1 = fmax3(a1, __uint_as_float(s[c >> 5][(c + 2) & 31]), __uint_as_float(s[c >> 5][(c + 3) & 31]));
+            a2 = fmax3(a2, __uint_as_float(s[c >> 5][(c + 4) & 31]), __uint_as_float(s[c >> 5][(c + 5) & 31]));
+            a3 = fmax3(a3, __uint_as_float(s[c >> 5][(c + 6) & 31]), __uint_as_float(s[c >> 5][(c + 7) & 31]));
+          }
+          mx = fmaxf(fmax3(a0, a1, a2), a3);
+        }
         const float m_new = fmaxf(m_run, mx * sl2);
         float alpha = 1.0f;
         bool resc = false;
@@ -297,66 +330,81 @@ __global__ void __launch_bounds__(kThreads, 1) partial_bf16_kernel(const __grid_
           resc = true;
         }
         const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
-        float sum = 0.0f;
+        // p = 2^(s * scale * log2 e - m) in packed pairs: kPolyPairsPer8 of every
+        // 8 pairs through the polynomial on the FMA pipe, the rest through the
+        // special-function unit. P goes back over the S row as bf16 pairs, 32
+        // columns at a time; the row sum runs in four packed chains.
+        const uint64_t sl2_2 = f2_pack(sl2, sl2);
+        const uint64_t negm_2 = f2_pack(-m_use, -m_use);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          const float pv = ex2(fmaf(__uint_as_float(s[c >> 5][c & 31]), sl2, -m_use));
-          s[c >> 5][c & 31] = __float_as_uint(pv);
-          sum += pv;
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int cc = 0; cc < 32; cc += 2) {
+            const int c = q4 * 32 + cc;
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[q4][cc]), __uint_as_float(s[q4][cc + 1])), sl2_2, negm_2);
+            uint64_t p2;
+            if (((c >> 1) & 7) < kPolyPairsPer8) {
+              p2 = exp2_poly_x2(x2);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              p2 = f2_pack(ex2(x0), ex2(x1));
+            }
+            float p0, p1;
+            f2_unpack(p2, p0, p1);
+            if (masked) {   // hidden keys contribute exactly zero (the polynomial leaves a tiny value)
+              if (c > lim) p0 = 0.0f;
+              if (c + 1 > lim) p1 = 0.0f;
+              p2 = f2_pack(p0, p1);
+            }
+            pk[cc >> 1] = pack_bf16x2(p0, p1);
+            acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], p2);
+          }
+          tmem_st16(s_col + q4 * 16, pk);
+        }
+        float sum;
+        {
+          const uint64_t t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+          float lo, hi;
+          f2_unpack(t, lo, hi);
+          sum = lo + hi;
         }
         l_run = l_run * alpha + sum;
-
-        if (it > 0) {
-          // PV of the previous tile must be done: it reads P and writes O.
-          if (!warp_wait(&bars[B_PV_DONE], (it - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-          if (__any_sync(0xffffffffu, resc)) {
-            tc_fence_after();
+        // O_x holds every earlier PV (see S_FULL above): rescale it in place if needed
+        if (it > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t o[32];
-              tmem_ld32(tmem + lane_base + kColO + c * 32, o);
-              tmem_ld_wait();
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(o_col + c * 32, o);
+            tmem_ld_wait();
 #pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-              tmem_st32(tmem + lane_base + kColO + c * 32, o);
-            }
-            tmem_st_wait();
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(o_col + c * 32, o);
           }
         }
-        // P row -> shared memory, bf16, 128-byte swizzled K-major layout
-#pragma unroll
-        for (int ch = 0; ch < 16; ++ch) {
-          const int c0 = ch * 8;
-          uint4 v4;
-          v4.x = pack_bf16x2(__uint_as_float(s[c0 >> 5][(c0 + 0) & 31]), __uint_as_float(s[c0 >> 5][(c0 + 1) & 31]));
-          v4.y = pack_bf16x2(__uint_as_float(s[c0 >> 5][(c0 + 2) & 31]), __uint_as_float(s[c0 >> 5][(c0 + 3) & 31]));
-          v4.z = pack_bf16x2(__uint_as_float(s[c0 >> 5][(c0 + 4) & 31]), __uint_as_float(s[c0 >> 5][(c0 + 5) & 31]));
-          v4.w = pack_bf16x2(__uint_as_float(s[c0 >> 5][(c0 + 6) & 31]), __uint_as_float(s[c0 >> 5][(c0 + 7) & 31]));
-          const int half = ch >> 3;
-          const int cc = ch & 7;
-          const uint32_t off = half * kHalfBytes + row * 128 + ((cc ^ (row & 7)) << 4);
-          *reinterpret_cast<uint4*>(sP + off) = v4;
-        }
-        fence_proxy_async_smem();
+        tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[B_P_FULL]);
+        if (lane == 0) mbar_arrive(&bars[B_P_FULL + x]);
       }
     }
 
     // ---------------------------------------------------------------- epilogue
     const int64_t out_row = ws.out_row0 + q_row0 + tok;
     const int head = kvh * group + (row & (group - 1));
-    if (ok && n_iter > 0) {
-      ok = warp_wait(&bars[B_PV_DONE], (n_iter - 1) & 1, abort_flag, p.status);
-      if (ok) {
+    bool done_ok = __all_sync(0xffffffffu, ok);
+    if (done_ok && n_iter > 0) {
+      done_ok = warp_wait(&bars[B_O_DONE + x], (n_iter - 1) & 1, abort_flag, p.status);
+      if (done_ok) {
         tc_fence_after();
         const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
         float* dst = p.o_part + (out_row * p.n_h + head) * HD;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem + lane_base + kColO + c * 32, o);
+          tmem_ld32(o_col + c * 32, o);
           tmem_ld_wait();
           if (row_valid) {
 #pragma unroll
@@ -368,12 +416,12 @@ __global__ void __launch_bounds__(kThreads, 1) partial_bf16_kernel(const __grid_
           }
         }
       }
-    } else if (n_iter == 0 && row_valid) {
+    } else if (done_ok && n_iter == 0 && row_valid) {
       float* dst = p.o_part + (out_row * p.n_h + head) * HD;
 #pragma unroll
       for (int i = 0; i < HD; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if (ok && row_valid) {
+    if (done_ok && row_valid) {
       const float lse = (l_run > 0.0f) ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
       p.lse_part[out_row * p.n_h + head] = lse;
     }
@@ -381,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1) partial_bf16_kernel(const __grid_
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
