@@ -43,6 +43,7 @@ EXPORTED = (
     "cp_status_string", "cp_abi_version", "cp_shard_plan", "cp_rank_ranges", "cp_ring_schedule",
     "cp_classify_pair", "cp_block_pairs", "cp_ring_comm_volume", "cp_workspace_size",
     "cp_reset_status", "cp_check_status", "cp_attn_partial", "cp_attn_merge", "cp_decode",
+    "cp_decode_static",
 )
 
 
@@ -97,6 +98,7 @@ def lib() -> ctypes.CDLL:
                                   P(cp_block), i32, vp, vp, i64, vp, sz, vp]),
         "cp_attn_merge": (i32, [vp, vp, i32, i64, i64, i32, i32, vp, i32, vp, vp]),
         "cp_decode": (i32, [vp, vp, vp, i32, vp, i32, i64, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]),
+        "cp_decode_static": (i32, [vp, vp, vp, i32, vp, i32, i64, i32, i32, i32, i32, f32, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -239,3 +241,14 @@ def cp_decode(q, k, v, kv_offsets, n_h: int, n_kv: int, n_splits: int, softmax_s
                            _ptr(out), _ptr(lse_out), _ptr(workspace),
                            int(workspace.numel() * workspace.element_size()), _stream(stream))
     _check("cp_decode", code)
+
+
+def cp_decode_static(q, k, v, kv_offsets, n_h: int, n_kv: int, n_splits: int, softmax_scale: float, out, lse_out,
+                     stream=None) -> None:
+    """cp_decode without a workspace, for callers that cannot allocate device
+    memory while decoding: the split partials use the library's fixed 32 MiB
+    array on the current device. Calls must not overlap on the GPU."""
+    code = lib().cp_decode_static(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(kv_offsets), int(q.shape[0]),
+                                  int(k.shape[0]), n_h, n_kv, int(q.shape[-1]), n_splits, float(softmax_scale),
+                                  _ptr(out), _ptr(lse_out), _stream(stream))
+    _check("cp_decode_static", code)

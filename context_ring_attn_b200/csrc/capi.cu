@@ -403,3 +403,55 @@ cp_status cp_decode(const void* q, const void* k, const void* v, cp_dtype dtype,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Split-KV decode without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory at the point where they decode:
+// code running inside a custom allocator or a memory pool that must not
+// re-enter itself, plugins handed only input and output buffers by a host
+// framework, and serving loops that forbid allocation after start-up. For
+// them the split partials live in one fixed array in the library's own device
+// memory (every GPU that loads the library holds it until the process exits).
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = 32ull << 20;  // 32 MiB per device
+static __device__ __align__(256) uint8_t g_decode_scratch[kStaticScratchBytes];
+
+// Device address of g_decode_scratch on each device. In host code the array's
+// name is only a stand-in; the address must be looked up with that device current.
+std::mutex g_scratch_mu;
+void* g_scratch_addr[64] = {nullptr};
+
+cp_status scratch_for_current_device(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CP_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || !ptr) return CP_ERR_CUDA;
+    g_scratch_addr[dev] = ptr;
+  }
+  *out = g_scratch_addr[dev];
+  return CP_OK;
+}
+
+}  // namespace
+
+extern "C" cp_status cp_decode_static(const void* q, const void* k, const void* v, cp_dtype dtype,
+                                      const int64_t* kv_offsets, int32_t batch, int64_t kv_rows, int32_t n_h,
+                                      int32_t n_kv, int32_t d, int32_t n_splits, float softmax_scale, void* out,
+                                      float* lse_out, void* cuda_stream) {
+  if (batch < 0 || n_h < 1 || d < 1 || n_splits < 1) return CP_ERR_INVALID_ARG;
+  const size_t need = cp_workspace_size(CP_OP_DECODE, batch, n_h, d, n_splits);
+  if (need > kStaticScratchBytes) return CP_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const cp_status st = scratch_for_current_device(&scratch);
+  if (st != CP_OK) return st;
+  // The status word must start at zero; the split partials are fully rewritten.
+  if (cudaMemsetAsync(scratch, 0, sizeof(uint32_t), static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+    return CP_ERR_CUDA;
+  return cp_decode(q, k, v, dtype, kv_offsets, batch, kv_rows, n_h, n_kv, d, n_splits, softmax_scale, out, lse_out,
+                   scratch, kStaticScratchBytes, cuda_stream);
+}

@@ -10,8 +10,9 @@
  * and the partials are combined by LSE weighting ("merge attention").
  *
  * Conventions shared by every entry point:
- *  - The caller owns and allocates every buffer. The library never allocates,
- *    frees or keeps device memory and holds no state between calls.
+ *  - The caller owns and allocates every buffer. The library never allocates
+ *    or frees device memory and holds no state between calls; the one
+ *    exception is the fixed scratch array behind cp_decode_static (below).
  *  - Tensors are row-major and token-major: Q [rows, N_H, D], K and V
  *    [rows, N_KV, D], partial outputs [rows, N_H, D] fp32, LSE [rows, N_H] fp32
  *    (natural logarithm of the sum of exp(scaled scores)).
@@ -230,6 +231,29 @@ cp_status cp_decode(const void* q, const void* k, const void* v, cp_dtype dtype,
                     const int64_t* kv_offsets, int32_t batch, int64_t kv_rows, int32_t n_h,
                     int32_t n_kv, int32_t d, int32_t n_splits, float softmax_scale, void* out,
                     float* lse_out, void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/* Split-KV decode for callers that cannot allocate device memory when they
+ * decode (code inside an allocator or memory pool, plugins that are given only
+ * their inputs and outputs, serving loops that forbid allocation after
+ * start-up). The method's pages have no counterpart to this entry point.
+ *
+ * Same arguments, results and limits as cp_decode, without the workspace: the
+ * split partials live in a fixed 32 MiB array in the library's device memory,
+ * which every GPU that loads the library holds until the process exits.
+ *  - Requests whose cp_workspace_size(CP_OP_DECODE, batch, n_h, d, n_splits)
+ *    exceeds 32 MiB are rejected with CP_ERR_WORKSPACE before any launch.
+ *  - The first call on a device looks up the array's device address for that
+ *    device (the device current at the call); make that first call before any
+ *    stream capture.
+ *  - Every call shares the one array, which keeps the last call's contents;
+ *    each call clears the status word it needs and rewrites every partial it
+ *    reads. Calls that overlap on the GPU (different streams without
+ *    ordering, or several host threads) race on the array.
+ *  - Nothing is allocated or freed. */
+cp_status cp_decode_static(const void* q, const void* k, const void* v, cp_dtype dtype,
+                           const int64_t* kv_offsets, int32_t batch, int64_t kv_rows, int32_t n_h,
+                           int32_t n_kv, int32_t d, int32_t n_splits, float softmax_scale, void* out,
+                           float* lse_out, void* cuda_stream);
 
 #ifdef __cplusplus
 }
