@@ -283,6 +283,10 @@ def run_ours(args, rank: int, world: int):
     e2e = run_e2e(args, q, k, v, out, lse, o_parts, lse_parts, ws, segs, n_ranks, n_h, n_kv, world, dev,
                   step_flops, barrier) if not args.no_e2e else None
     decode = run_decode(args, dev) if not args.no_decode else None
+    secondary = {}
+    if not args.no_secondary:
+        for name in ("persistent_kv", "varlen_prefill"):
+            secondary[name] = run_secondary(args, dev, name)
 
     if rank != 0:
         return
@@ -315,6 +319,8 @@ def run_ours(args, rank: int, world: int):
     }
     if decode:
         line["decode"] = decode
+    if secondary:
+        line["workloads"] = secondary
     if not args.no_cpu_baseline:
         f, s, n = oracle_sample(args.cpu_seconds)
         line["cpu_baseline"] = {
@@ -378,6 +384,107 @@ def run_e2e(args, q, k, v, out, lse, o_parts, lse_parts, ws, segs, n_ranks, n_h,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
+def run_secondary(args, dev, name: str):
+    """The other prefill workloads, each a full ring schedule per step:
+    persistent-KV partial prefill (T=4096 new over P=126976 cached, 128/8
+    heads, pass-Q, 8-way merge) and the varlen batch (8 sequences, 262144
+    tokens, 128/8 heads, pass-KV, running 2-way merges to bound memory)."""
+    import torch
+
+    from context_ring_attn_b200 import binding as B
+    from context_ring_attn_b200 import ring, synth
+
+    w = synth.WORKLOADS[name]
+    n_h, n_kv, d, n = w["n_h"], w["n_kv"], w["d"], w["n_ranks"]
+    scale = 1.0 / math.sqrt(d)
+    if name == "persistent_kv":
+        t, p = w["t"], w["p"]
+        q_segs = [ring.Segment(t, 0, p, 0)]
+        kv_segs = [ring.Segment(p, 0, 0, 0), ring.Segment(t, p, p, 0)]
+        kv_rows, variant, merge = p + t, B.CP_PASS_Q, "final"
+        desc = {"T": t, "P": p, "ring": "pass-Q", "merge": "final 8-way"}
+    else:
+        lens = synth.varlen_lengths(w["seed"], w["n_seq"], w["total"])
+        t = w["total"]
+        starts = np.concatenate([[0], np.cumsum(lens)[:-1]]).astype(np.int64)
+        q_segs = kv_segs = [ring.Segment(int(ln), int(s0), 0, i) for i, (ln, s0) in enumerate(zip(lens, starts))]
+        kv_rows, variant, merge = t, B.CP_PASS_KV, "running"
+        desc = {"seq_lens": [int(x) for x in lens], "ring": "pass-KV", "merge": "running 2-way"}
+    q = synth.device_rows(w["seed"], synth.TENSOR_Q, t, (n_h, d), w["std"], "bf16", dev)
+    k = synth.device_rows(w["seed"], synth.TENSOR_K, kv_rows, (n_kv, d), w["std"], "bf16", dev)
+    v = synth.device_rows(w["seed"], synth.TENSOR_V, kv_rows, (n_kv, d), w["std"], "bf16", dev)
+    n_bufs = n if merge == "final" else 2
+    o_parts, lse_parts = ring.partial_buffers(t, n_h, d, n_bufs, dev)
+    out = torch.empty((t, n_h, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((t, n_h), dtype=torch.float32, device=dev)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sched0 = ring.RingSchedule(q_segs, kv_segs, n, variant)
+    pairs = sched0.pairs(True)
+    step_flops = 4.0 * d * n_h * pairs
+    ev_part, ev_merge = [], []
+
+    def step(record):
+        sched = ring.RingSchedule(q_segs, kv_segs, n, variant)
+        for s_ in range(n):
+            target = (lambda pt: pt) if merge == "final" else (lambda _pt, _t=(0 if s_ == 0 else 1): _t)
+            blocks = sched.step_blocks(s_, t, part_of=target)
+            e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) if record else None
+            if e:
+                e[0].record(stream)
+            B.cp_attn_partial(q, k, v, n_h, n_kv, scale, True, sched.ranges, sched.n_ranges, blocks, n, o_parts,
+                              lse_parts, ws)
+            if e:
+                e[1].record(stream)
+                ev_part.append(e)
+            if merge == "running" and s_ > 0:
+                last = s_ == n - 1
+                e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) if record else None
+                if e:
+                    e[0].record(stream)
+                B.cp_attn_merge(o_parts, lse_parts, 2, t, t, n_h, d, out if last else o_parts,
+                                lse if last else lse_parts)
+                if e:
+                    e[1].record(stream)
+                    ev_merge.append((e, 2 * t * n_h * (d + 1) * 4 + t * n_h * ((2 * d + 4) if last else (d + 1) * 4)))
+        if merge == "final":
+            e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) if record else None
+            if e:
+                e[0].record(stream)
+            B.cp_attn_merge(o_parts, lse_parts, n, t, t, n_h, d, out, lse)
+            if e:
+                e[1].record(stream)
+                ev_merge.append((e, n * t * n_h * (d + 1) * 4 + t * n_h * (2 * d + 4)))
+
+    for _ in range(3):
+        step(False)
+    torch.cuda.synchronize()
+    steps = max(2, args.steps // 4)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step(True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    B.cp_check_status(ws)
+    ms = e0.elapsed_time(e1) / steps
+    part_ms = sum(a.elapsed_time(b) for a, b in ev_part) / steps
+    merge_ms = sum(a.elapsed_time(b) for (a, b), _ in ev_merge) / steps
+    merge_bytes = sum(nb for _, nb in ev_merge) / steps
+    peaks, kind = load_peaks()
+    peak_t = float(peaks["bf16_tflops_sustained"])
+    res = {"value": step_flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms, "steps": steps,
+           "flops_per_step": step_flops, "N_H": n_h, "N_KV": n_kv, "cp_ranks": n, **desc,
+           "partial_tflops": step_flops / (part_ms * 1e-3) / 1e12,
+           "partial_frac": step_flops / (part_ms * 1e-3) / 1e12 / peak_t,
+           "merge_gbs": merge_bytes / (merge_ms * 1e-3) / 1e9,
+           "merge_frac_hbm": merge_bytes / (merge_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
+           "peak_kind": f"bf16_tflops_sustained / hbm_gbs ({kind})"}
+    del q, k, v, o_parts, lse_parts, out, lse
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_decode(args, dev):
     """Split-KV decode: 32 requests, 16 heads on 1 KV head, 256 splits; GB/s
     of K/V read (each byte once)."""
@@ -434,6 +541,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the persistent-KV and varlen workloads")
     ap.add_argument("--only-decode", action="store_true", help="time the split-KV decode workload alone")
     ap.add_argument("--tokens", type=int, default=0,
                     help="shorter sequence for profiling captures (default: the full 131072)")
