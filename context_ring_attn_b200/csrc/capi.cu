@@ -399,7 +399,10 @@ cp_status cp_decode(const void* q, const void* k, const void* v, cp_dtype dtype,
   dim3 grid(n_splits, batch * n_kv);
   dec::decode_split_kernel<<<grid, dec::kThreads, dec::kSmemBytes, stream>>>(p);
   if (last_cuda_status() != CP_OK) return CP_ERR_CUDA;
-  return cp_attn_merge(o_ws, l_ws, n_splits, batch, batch, n_h, d, out, CP_BF16, lse_out, cuda_stream);
+  const int64_t n_rowheads = static_cast<int64_t>(batch) * n_h;
+  dec::decode_merge_kernel<<<static_cast<unsigned>(n_rowheads), dec::kMergeThreads, 0, stream>>>(
+      o_ws, l_ws, n_splits, n_rowheads, static_cast<__nv_bfloat16*>(out), lse_out);
+  return last_cuda_status();
 }
 
 }  // extern "C"

@@ -290,5 +290,84 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const __grid_
   }
 }
 
+// Merge of the split partials of one (request, head) per CTA: the 8 warps take
+// every 8th split, each keeps an online (max, sum, O) over its splits with
+// float4 loads eight splits deep, and the eight results are combined in shared
+// memory. Same formula as the generic merge (LSE weighting, -inf splits weigh
+// 0); more warps per row so the 256 splits stream at full bandwidth.
+constexpr int kMergeThreads = 256;
+constexpr int kMergeUnroll = 8;
+
+__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const float* __restrict__ o_parts,
+                                                                      const float* __restrict__ lse_parts,
+                                                                      int n_splits, int64_t n_rowheads,
+                                                                      __nv_bfloat16* out, float* lse_out) {
+  __shared__ float sm_m[8], sm_l[8];
+  __shared__ float4 sm_o[8][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t rh = blockIdx.x;
+  const int64_t o_stride = n_rowheads * 128;   // floats between splits
+  float m = -INFINITY, l = 0.0f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j0 = warp; j0 < n_splits; j0 += 8 * kMergeUnroll) {
+    float4 x[kMergeUnroll];
+    float lj[kMergeUnroll];
+#pragma unroll
+    for (int u = 0; u < kMergeUnroll; ++u) {
+      const int j = j0 + u * 8;
+      lj[u] = -INFINITY;
+      x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j < n_splits) {
+        lj[u] = __ldg(lse_parts + j * n_rowheads + rh);
+        x[u] = __ldcs(reinterpret_cast<const float4*>(o_parts + j * o_stride + rh * 128) + lane);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kMergeUnroll; ++u) {
+      if (lj[u] == -INFINITY) continue;
+      const float m_new = fmaxf(m, lj[u]);
+      const float so = __expf(m - m_new);   // 0 when m was -inf
+      const float wj = __expf(lj[u] - m_new);
+      l = l * so + wj;
+      acc.x = fmaf(wj, x[u].x, acc.x * so);
+      acc.y = fmaf(wj, x[u].y, acc.y * so);
+      acc.z = fmaf(wj, x[u].z, acc.z * so);
+      acc.w = fmaf(wj, x[u].w, acc.w * so);
+      m = m_new;
+    }
+  }
+  if (lane == 0) {
+    sm_m[warp] = m;
+    sm_l[warp] = l;
+  }
+  sm_o[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) M = fmaxf(M, sm_m[w]);
+    float L = 0.0f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        const float sc = expf(sm_m[w] - M);   // 0 for warps that saw no split
+        L += sm_l[w] * sc;
+        const float4 a = sm_o[w][lane];
+        o.x = fmaf(sc, a.x, o.x);
+        o.y = fmaf(sc, a.y, o.y);
+        o.z = fmaf(sc, a.z, o.z);
+        o.w = fmaf(sc, a.w, o.w);
+      }
+    }
+    const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
+    uint2 u;
+    u.x = pack_bf16x2(o.x * inv, o.y * inv);
+    u.y = pack_bf16x2(o.z * inv, o.w * inv);
+    *reinterpret_cast<uint2*>(out + rh * 128 + lane * 4) = u;
+    if (lse_out && lane == 0) lse_out[rh] = (L > 0.0f) ? M + logf(L) : -INFINITY;
+  }
+}
+
 }  // namespace dec
 }  // namespace cpk
