@@ -528,7 +528,7 @@ def run_decode(args, dev):
     return {"value": gbs, "unit": "GB/s", "ms": ms, "kv_bytes": kv_bytes, "batch": b, "n_splits": ns,
             "frac_hbm": gbs / float(peaks["hbm_gbs"]), "peak": float(peaks["hbm_gbs"]),
             "peak_kind": f"hbm_gbs ({kind})", "l2": "256 MB buffer written between iterations",
-            "note": "split kernel + 256-way merge, median of iterations"}
+            "note": "balanced split kernel (8 ranges per SM) + per-head merge, median of iterations"}
 
 
 def main():

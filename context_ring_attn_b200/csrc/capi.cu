@@ -195,6 +195,23 @@ constexpr size_t kStatusBytes = 256;
 
 inline size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Ranges of the flattened decode keys (one per warp of the persistent split
+// grid): 8 per SM of the current device, at most n_splits per (request, KV head).
+cp_status decode_ranges(int32_t n_splits, int32_t batch, int32_t n_kv, int32_t* n_warps) {
+  int n_sm = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return CP_ERR_CUDA;
+  const int64_t want = (static_cast<int64_t>(n_splits) * batch * n_kv + 7) / 8;
+  *n_warps = static_cast<int32_t>(std::max<int64_t>(1, std::min<int64_t>(n_sm, want)) * 8);
+  return CP_OK;
+}
+
+// Workspace bytes cp_decode uses with n_warps ranges (never above cp_workspace_size).
+size_t decode_ws_bytes(int32_t n_warps, int32_t batch, int32_t n_h, int32_t n_kv, int32_t d) {
+  const size_t part = (static_cast<size_t>(n_warps) + static_cast<size_t>(batch) * n_kv) * (n_h / n_kv);
+  return kStatusBytes + round256(part * d * 4) + round256(part * 4);
+}
+
 }  // namespace
 
 extern "C" {
@@ -202,7 +219,9 @@ extern "C" {
 size_t cp_workspace_size(cp_op op, int64_t rows, int32_t n_h, int32_t d, int32_t n_splits) {
   if (op == CP_OP_DECODE) {
     if (rows < 0 || n_h < 1 || d < 1 || n_splits < 1) return kStatusBytes;
-    const size_t part = static_cast<size_t>(n_splits) * static_cast<size_t>(rows) * static_cast<size_t>(n_h);
+    // at most n_splits*batch*n_kv + 7 ranges + batch*n_kv pairs, G = n_h/n_kv rows each
+    const size_t part = (static_cast<size_t>(n_splits) + 1) * static_cast<size_t>(rows) * static_cast<size_t>(n_h) +
+                        7 * static_cast<size_t>(n_h);
     return kStatusBytes + round256(part * static_cast<size_t>(d) * 4) + round256(part * 4);
   }
   return kStatusBytes;
@@ -371,10 +390,13 @@ cp_status cp_decode(const void* q, const void* k, const void* v, cp_dtype dtype,
   if (dtype != CP_BF16 || d != 128 || group > 16 || (16 % group) != 0) return CP_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 8) || !aligned(kv_offsets, 8))
     return CP_ERR_INVALID_ARG;
-  if (!workspace || !aligned(workspace, 256) || ws_bytes < cp_workspace_size(CP_OP_DECODE, batch, n_h, d, n_splits))
-    return CP_ERR_WORKSPACE;
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < decode_ws_bytes(dec::kWarps, batch, n_h, n_kv, d))
+    return CP_ERR_WORKSPACE;   // below what even the smallest grid needs
   if (batch == 0) return CP_OK;
-  const size_t part = static_cast<size_t>(n_splits) * batch * n_h;
+  int32_t n_warps = 0;
+  if (decode_ranges(n_splits, batch, n_kv, &n_warps) != CP_OK) return CP_ERR_CUDA;
+  if (ws_bytes < decode_ws_bytes(n_warps, batch, n_h, n_kv, d)) return CP_ERR_WORKSPACE;
+  const size_t part = (static_cast<size_t>(n_warps) + static_cast<size_t>(batch) * n_kv) * group;
   float* o_ws = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
   float* l_ws = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes + round256(part * d * 4));
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
@@ -391,17 +413,17 @@ cp_status cp_decode(const void* q, const void* k, const void* v, cp_dtype dtype,
   p.n_h = n_h;
   p.n_kv = n_kv;
   p.group = group;
-  p.n_splits = n_splits;
+  p.n_warps = n_warps;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   if (cudaFuncSetAttribute(dec::decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            dec::kSmemBytes) != cudaSuccess)
     return CP_ERR_CUDA;
-  dim3 grid(n_splits, batch * n_kv);
-  dec::decode_split_kernel<<<grid, dec::kThreads, dec::kSmemBytes, stream>>>(p);
+  // persistent: up to one CTA per SM, each warp streaming one range of the flattened keys
+  dec::decode_split_kernel<<<static_cast<unsigned>(n_warps / dec::kWarps), dec::kThreads, dec::kSmemBytes, stream>>>(p);
   if (last_cuda_status() != CP_OK) return CP_ERR_CUDA;
   const int64_t n_rowheads = static_cast<int64_t>(batch) * n_h;
   dec::decode_merge_kernel<<<static_cast<unsigned>(n_rowheads), dec::kMergeThreads, 0, stream>>>(
-      o_ws, l_ws, n_splits, n_rowheads, static_cast<__nv_bfloat16*>(out), lse_out);
+      p, static_cast<__nv_bfloat16*>(out), lse_out);
   return last_cuda_status();
 }
 
@@ -446,9 +468,11 @@ extern "C" cp_status cp_decode_static(const void* q, const void* k, const void* 
                                       const int64_t* kv_offsets, int32_t batch, int64_t kv_rows, int32_t n_h,
                                       int32_t n_kv, int32_t d, int32_t n_splits, float softmax_scale, void* out,
                                       float* lse_out, void* cuda_stream) {
-  if (batch < 0 || n_h < 1 || d < 1 || n_splits < 1) return CP_ERR_INVALID_ARG;
-  const size_t need = cp_workspace_size(CP_OP_DECODE, batch, n_h, d, n_splits);
-  if (need > kStaticScratchBytes) return CP_ERR_WORKSPACE;
+  if (batch < 0 || n_h < 1 || n_kv < 1 || d < 1 || n_splits < 1 || n_h % n_kv) return CP_ERR_INVALID_ARG;
+  if (n_splits > dec::kMaxSplits) return CP_ERR_UNSUPPORTED;
+  int32_t n_warps = 0;
+  if (decode_ranges(n_splits, batch, n_kv, &n_warps) != CP_OK) return CP_ERR_CUDA;
+  if (decode_ws_bytes(n_warps, batch, n_h, n_kv, d) > kStaticScratchBytes) return CP_ERR_WORKSPACE;
   void* scratch = nullptr;
   const cp_status st = scratch_for_current_device(&scratch);
   if (st != CP_OK) return st;

@@ -1,18 +1,26 @@
 // Split-KV decode: one query token per request against its whole KV cache,
-// the keys cut into n_splits splits, one partial (O, LSE) per split, then the
-// LSE merge ("Context Parallelism for Scalable Million-Token Inference",
-// section 5 software stack: Flash Decoding with 256 splits; decode itself per
-// "Context Parallelism과 Expert Parallelism" section 5.2).
+// the keys cut into splits, one partial (O, LSE) per split, then the LSE merge
+// ("Context Parallelism for Scalable Million-Token Inference", section 5
+// software stack: Flash Decoding; decode itself per "Context Parallelism과
+// Expert Parallelism" section 5.2).
 //
 // The work is HBM-bound (every K/V byte is read once; 16 flop per byte with
 // 16 query heads per KV head), so the design goal is streaming K/V at full
-// bandwidth: each CTA (4 warps) owns one (split, request, KV head), streams
-// 64-key chunks of K and V with 16-byte cp.async copies (fully coalesced rows
-// of 256 bytes) into a 3-stage shared-memory ring with a 16-byte-chunk XOR
-// swizzle, and each warp takes 16 keys of every chunk. All G <= 16 query
-// heads of the KV head share each K/V load: they form the 16 rows of
-// m16n8k16 bf16 MMAs (S = q K^T and O += P V with P kept in registers).
-// At the end the four warps' (max, sum, O) are combined in shared memory.
+// bandwidth with the least fixed cost and no tail. The splits are cut over
+// the whole batch: the keys of all (request, KV head) pairs, in order, form
+// one flattened sequence of Kt = n_kv * (offsets[B] - offsets[0]) keys, and
+// warp w of the persistent grid of W warps owns the range
+// [w*Kt/W, (w+1)*Kt/W). Every warp thus streams the same number of keys
+// (within one key), whatever the mix of request lengths, and writes one
+// partial per (request, KV head) its range overlaps: about W + B*n_kv
+// partials in all. Warp w's partial for pair bg lands in slot w + bg, which is
+// unique because both the ranges and the pairs are in flattened order.
+//
+// Each warp works alone: a private 3-stage ring of 16-key steps of K and V in
+// shared memory, filled by 16-byte cp.async copies (rows of 256 bytes, fully
+// coalesced) that run ahead across pair boundaries. All G <= 16 query heads
+// of the KV head share every K/V load: they are the 16 rows of m16n8k16 bf16
+// MMAs (S = q K^T, then O += P V with P kept in registers).
 #pragma once
 
 #include "common.cuh"
@@ -20,12 +28,14 @@
 namespace cpk {
 namespace dec {
 
-constexpr int kThreads = 128;
-constexpr int kChunk = 64;       // keys per pipeline stage
-constexpr int kStages = 3;
-constexpr int kRowBytes = 256;   // 128 bf16
-constexpr int kStageBytes = 2 * kChunk * kRowBytes;  // K + V
-constexpr int kSmemBytes = kStages * kStageBytes;    // 96 KB
+constexpr int kWarps = 8;                 // warps per CTA, one CTA per SM
+constexpr int kThreads = kWarps * 32;
+constexpr int kStepKeys = 16;             // keys per pipeline step of a warp
+constexpr int kStages = 3;                // steps in flight per warp
+constexpr int kRowBytes = 256;            // 128 bf16
+constexpr int kStepBytes = 2 * kStepKeys * kRowBytes;   // K + V of one step: 8 KB
+constexpr int kWarpBytes = kStages * kStepBytes;        // 24 KB per warp
+constexpr int kSmemBytes = kWarps * kWarpBytes;         // 192 KB
 constexpr int kMaxSplits = 1024;
 
 struct Params {
@@ -34,14 +44,14 @@ struct Params {
   const __nv_bfloat16* v;
   const int64_t* offsets;
   int64_t kv_rows;
-  float* o_part;   // [n_splits][batch][n_h][128]
-  float* lse_part; // [n_splits][batch][n_h]
+  float* o_part;   // [slot][G][128], slot = warp + pair
+  float* lse_part; // [slot][G]
   uint32_t* status;
   int32_t batch;
   int32_t n_h;
   int32_t n_kv;
   int32_t group;
-  int32_t n_splits;
+  int32_t n_warps; // W: warps of the split grid = ranges of the flattened keys
   float scale_log2;
 };
 
@@ -74,252 +84,331 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// byte offset of 16-byte chunk c of key row r inside a K or V stage
+// byte offset of 16-byte chunk c of key row r inside a K or V step
 __device__ __forceinline__ uint32_t swz(int r, int c) { return r * kRowBytes + ((c ^ (r & 7)) << 4); }
 
-__global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const __grid_constant__ Params p) {
+// floor(x / y) for 0 <= x < 2^53, 0 < y < 2^53, exactly: the double quotient
+// is correctly rounded, so its truncation is the true quotient or one above it
+// (when x / y lies just below an integer); one integer check settles it.
+__device__ __forceinline__ int64_t floordiv(int64_t x, int64_t y) {
+  int64_t q = static_cast<int64_t>(static_cast<double>(x) / static_cast<double>(y));
+  if (q * y > x) --q;
+  return q;
+}
+
+// First key of range w of the flattened sequence of kt keys cut into n ranges.
+__device__ __forceinline__ int64_t range_start(int64_t w, int64_t kt, int64_t n) { return floordiv(w * kt, n); }
+
+// The range holding flattened key x (0 <= x < kt): the largest w with start(w) <= x.
+__device__ __forceinline__ int64_t range_of(int64_t x, int64_t kt, int64_t n) {
+  const int64_t w = floordiv((x + 1) * n - 1, kt);
+  return w < n - 1 ? w : n - 1;
+}
+
+// Part of one warp's range inside one (request, KV head) pair.
+struct Piece {
+  int64_t row0;  // first K/V row
+  int n_keys;
+  int b, g, bg;
+};
+
+// Walks the pairs that overlap [a, e) in flattened order. Every pair it looks
+// at is checked (rows inside [0, kv_rows)), so the walk stays in bounds even
+// for offsets that break the non-decreasing contract; the merge reports those.
+struct Walker {
+  int bg;        // next pair to look at
+  int64_t a, e;  // the range
+  int64_t o0;    // offsets[0]
+
+  __device__ __forceinline__ void init(const Params& p, int64_t a_, int64_t e_, int64_t o0_) {
+    a = a_;
+    e = e_;
+    o0 = o0_;
+    int lo = 0, hi = p.batch - 1;   // last request whose first flattened key is <= a
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if ((p.offsets[mid] - o0) * p.n_kv <= a) lo = mid;
+      else hi = mid - 1;
+    }
+    const int64_t base = p.offsets[lo], len = p.offsets[lo + 1] - base;
+    int64_t g = 0;
+    if (len > 0) {
+      g = (a - (base - o0) * p.n_kv) / len;
+      g = g < 0 ? 0 : (g >= p.n_kv ? p.n_kv - 1 : g);
+    }
+    bg = lo * p.n_kv + static_cast<int>(g);
+  }
+
+  // next non-empty piece; false once the range is done
+  __device__ __forceinline__ bool next(const Params& p, Piece& t) {
+    const int n_bg = p.batch * p.n_kv;
+    while (bg < n_bg) {
+      const int cur = bg++;
+      const int b = cur / p.n_kv;
+      const int g = cur - b * p.n_kv;
+      const int64_t base = p.offsets[b], end = p.offsets[b + 1];
+      if (!(base >= o0 && end >= base && end <= p.kv_rows)) continue;
+      const int64_t len = end - base;
+      const int64_t vs = (base - o0) * p.n_kv + g * len;
+      if (vs >= e) {
+        bg = n_bg;
+        return false;
+      }
+      const int64_t lo = a > vs ? a : vs;
+      const int64_t hi = e < vs + len ? e : vs + len;
+      if (hi > lo) {
+        t.row0 = base + (lo - vs);
+        t.n_keys = static_cast<int>(hi - lo);
+        t.b = b;
+        t.g = g;
+        t.bg = cur;
+        return true;
+      }
+    }
+    return false;
+  }
+};
+
+__global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int split = blockIdx.x;
-  const int b = blockIdx.y / p.n_kv;
-  const int g = blockIdx.y - b * p.n_kv;
-
-  const int64_t base = p.offsets[b];
-  const int64_t end = p.offsets[b + 1];
-  const bool offsets_ok = base >= 0 && end >= base && end <= p.kv_rows;
-  if (!offsets_ok && threadIdx.x == 0) atomicOr(p.status, kStatusInternal);
-  const int64_t len = offsets_ok ? end - base : 0;
-  const int64_t lo = (static_cast<int64_t>(split) * len) / p.n_splits;
-  const int64_t hi = (static_cast<int64_t>(split + 1) * len) / p.n_splits;
-  const int n_keys = static_cast<int>(hi - lo);
-  const int n_chunks = (n_keys + kChunk - 1) / kChunk;
-  const int64_t key0 = base + lo;
-
-  const uint32_t s_base = smem_u32(smem);
-  const int row_stride = p.n_kv * 128;  // elements between consecutive keys
-
-  auto load_chunk = [&](int c, int stage) {
-    const uint32_t sk = s_base + stage * kStageBytes;
-    const uint32_t sv = sk + kChunk * kRowBytes;
-#pragma unroll
-    for (int i = 0; i < (kChunk * 16) / kThreads; ++i) {
-      const int e = threadIdx.x + i * kThreads;  // 16-byte chunk index within the 64x256B tile
-      const int r = e >> 4;
-      const int cc = e & 15;
-      const int kr = c * kChunk + r;
-      const bool in = kr < n_keys;
-      const int64_t row = in ? key0 + kr : 0;
-      const size_t off = static_cast<size_t>(row) * row_stride + g * 128 + cc * 8;
-      cp_async16(sk + swz(r, cc), p.k + off, in ? 16u : 0u);
-      cp_async16(sv + swz(r, cc), p.v + off, in ? 16u : 0u);
-    }
-  };
-
-#pragma unroll
-  for (int s = 0; s < kStages - 1; ++s) {
-    if (s < n_chunks) load_chunk(s, s);
-    cp_async_commit();
-  }
-
-  // Q fragments: rows = query heads of the group (rows >= G are zero), 8 k-steps of 16 dims.
-  const int gr = lane >> 2;  // fragment row
-  const int tq = lane & 3;   // fragment column pair
-  uint32_t qa[8][4];
-  {
-    const __nv_bfloat16* qb = p.q + (static_cast<size_t>(b) * p.n_h + g * p.group) * 128;
-    const bool r0 = gr < p.group, r1 = gr + 8 < p.group;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const int c0 = ks * 16 + tq * 2;
-      qa[ks][0] = r0 ? *reinterpret_cast<const uint32_t*>(qb + gr * 128 + c0) : 0u;
-      qa[ks][1] = r1 ? *reinterpret_cast<const uint32_t*>(qb + (gr + 8) * 128 + c0) : 0u;
-      qa[ks][2] = r0 ? *reinterpret_cast<const uint32_t*>(qb + gr * 128 + c0 + 8) : 0u;
-      qa[ks][3] = r1 ? *reinterpret_cast<const uint32_t*>(qb + (gr + 8) * 128 + c0 + 8) : 0u;
-    }
-  }
-
-  float o[16][4];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.0f;
-  float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 units) of rows gr, gr+8
-  float l0 = 0.0f, l1 = 0.0f;            // thread-partial running sums
+  const int gw = blockIdx.x * kWarps + warp;
+  const uint32_t ring = smem_u32(smem) + warp * kWarpBytes;
+  const int row_stride = p.n_kv * 128;   // elements between consecutive keys
   const float sl2 = p.scale_log2;
+  const int gr = lane >> 2;  // fragment row (query head in the group)
+  const int tq = lane & 3;   // fragment column pair
 
-  for (int c = 0; c < n_chunks; ++c) {
-    cp_async_wait<kStages - 2>();
-    __syncthreads();
-    if (c + kStages - 1 < n_chunks) load_chunk(c + kStages - 1, (c + kStages - 1) % kStages);
+  const int64_t o0 = p.offsets[0];
+  const int64_t oB = p.offsets[p.batch];
+  if (!(o0 >= 0 && oB >= o0 && oB <= p.kv_rows)) return;   // reported by the merge
+  const int64_t kt = (oB - o0) * p.n_kv;
+  if (kt == 0) return;
+  const int64_t a = range_start(gw, kt, p.n_warps);
+  const int64_t e = range_start(gw + 1, kt, p.n_warps);
+
+  // ---- loader: walks the same pieces and 16-key steps as the compute loop
+  Walker lw;
+  lw.init(p, a, e, o0);
+  Piece lp;
+  bool l_more = lw.next(p, lp);
+  int l_step = 0;
+  int l_slot = 0;
+  auto issue_step = [&]() {   // copies of one step, or nothing once the range is done
+    if (l_more) {
+      const uint32_t sk = ring + l_slot * kStepBytes;
+      const uint32_t sv = sk + kStepKeys * kRowBytes;
+#pragma unroll
+      for (int i = 0; i < (kStepKeys * 16) / 32; ++i) {
+        const int c = lane + i * 32;   // 16-byte chunk of the 16 x 256-byte step
+        const int r = c >> 4;
+        const int cc = c & 15;
+        const int kr = l_step * kStepKeys + r;
+        const bool in = kr < lp.n_keys;
+        const int64_t row = in ? lp.row0 + kr : 0;
+        const size_t off = static_cast<size_t>(row) * row_stride + lp.g * 128 + cc * 8;
+        cp_async16(sk + swz(r, cc), p.k + off, in ? 16u : 0u);
+        cp_async16(sv + swz(r, cc), p.v + off, in ? 16u : 0u);
+      }
+      l_slot = (l_slot + 1) % kStages;
+      if (++l_step * kStepKeys >= lp.n_keys) {
+        l_step = 0;
+        l_more = lw.next(p, lp);
+      }
+    }
     cp_async_commit();
+  };
+#pragma unroll
+  for (int s = 0; s < kStages - 1; ++s) issue_step();
 
-    const uint32_t sk = s_base + (c % kStages) * kStageBytes;
-    const uint32_t sv = sk + kChunk * kRowBytes;
-    const int kw = warp * 16;  // this warp's 16 keys of the chunk
-
-    // S = Q K^T for 16 keys: two n-tiles of 8 keys
-    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  Walker cw;
+  cw.init(p, a, e, o0);
+  Piece t;
+  int c_slot = 0;
+  while (cw.next(p, t)) {
+    const size_t prow = static_cast<size_t>(gw + t.bg) * p.group;   // first partial row of this piece
+    // Q fragments: rows = query heads of the group (rows >= G are zero), 8 k-steps of 16 dims
+    uint32_t qa[8][4];
     {
-      const int mi = lane >> 3, rr = lane & 7;
-      const int key = kw + (mi >> 1) * 8 + rr;
+      const __nv_bfloat16* qb = p.q + (static_cast<size_t>(t.b) * p.n_h + t.g * p.group) * 128;
+      const bool r0 = gr < p.group, r1 = gr + 8 < p.group;
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(sk + swz(key, ks * 2 + (mi & 1)), b0, b1, b2, b3);
-        mma16816(s[0], qa[ks], b0, b1);
-        mma16816(s[1], qa[ks], b2, b3);
+        const int c0 = ks * 16 + tq * 2;
+        qa[ks][0] = r0 ? *reinterpret_cast<const uint32_t*>(qb + gr * 128 + c0) : 0u;
+        qa[ks][1] = r1 ? *reinterpret_cast<const uint32_t*>(qb + (gr + 8) * 128 + c0) : 0u;
+        qa[ks][2] = r0 ? *reinterpret_cast<const uint32_t*>(qb + gr * 128 + c0 + 8) : 0u;
+        qa[ks][3] = r1 ? *reinterpret_cast<const uint32_t*>(qb + (gr + 8) * 128 + c0 + 8) : 0u;
       }
     }
-    // mask keys past the split end
-    const int valid = n_keys - c * kChunk - kw;  // keys of this warp's 16 that exist
+    float o[16][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const int col = nt * 8 + tq * 2;
-      if (col >= valid) { s[nt][0] = -INFINITY; s[nt][2] = -INFINITY; }
-      if (col + 1 >= valid) { s[nt][1] = -INFINITY; s[nt][3] = -INFINITY; }
-    }
-    float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
-    float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float n0 = fmaxf(m0, mx0 * sl2);
-    const float n1 = fmaxf(m1, mx1 * sl2);
-    const float u0 = (n0 == -INFINITY) ? 0.0f : n0;
-    const float u1 = (n1 == -INFINITY) ? 0.0f : n1;
-    const float a0 = ex2(m0 - u0);
-    const float a1 = ex2(m1 - u1);
-    m0 = n0;
-    m1 = n1;
-    float pr[2][4];
+    for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.0f;
+    float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 units) of rows gr, gr+8
+    float l0 = 0.0f, l1 = 0.0f;            // thread-partial running sums
+    const int n_steps = (t.n_keys + kStepKeys - 1) / kStepKeys;
+
+    for (int st = 0; st < n_steps; ++st) {
+      cp_async_wait<kStages - 2>();
+      __syncwarp();
+      issue_step();
+      const uint32_t sk = ring + c_slot * kStepBytes;
+      const uint32_t sv = sk + kStepKeys * kRowBytes;
+      c_slot = (c_slot + 1) % kStages;
+
+      // S = Q K^T for 16 keys: two n-tiles of 8 keys
+      float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      {
+        const int mi = lane >> 3, rr = lane & 7;
+        const int key = (mi >> 1) * 8 + rr;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      pr[nt][0] = ex2(fmaf(s[nt][0], sl2, -u0));
-      pr[nt][1] = ex2(fmaf(s[nt][1], sl2, -u0));
-      pr[nt][2] = ex2(fmaf(s[nt][2], sl2, -u1));
-      pr[nt][3] = ex2(fmaf(s[nt][3], sl2, -u1));
-    }
-    l0 = l0 * a0 + pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1];
-    l1 = l1 * a1 + pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      o[j][0] *= a0;
-      o[j][1] *= a0;
-      o[j][2] *= a1;
-      o[j][3] *= a1;
-    }
-    uint32_t pa[4];
-    pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
-    pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
-    pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
-    pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
-    // O += P V: 16 d-tiles of 8, two per transposed ldmatrix.x4
-    {
-      const int mi = lane >> 3, rr = lane & 7;
-      const int key = kw + (mi & 1) * 8 + rr;
-#pragma unroll
-      for (int j = 0; j < 16; j += 2) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(sv + swz(key, j + (mi >> 1)), b0, b1, b2, b3);
-        mma16816(o[j], pa, b0, b1);
-        mma16816(o[j + 1], pa, b2, b3);
+        for (int ks = 0; ks < 8; ++ks) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(sk + swz(key, ks * 2 + (mi & 1)), b0, b1, b2, b3);
+          mma16816(s[0], qa[ks], b0, b1);
+          mma16816(s[1], qa[ks], b2, b3);
+        }
       }
+      // mask keys past the piece end
+      const int valid = t.n_keys - st * kStepKeys;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int col = nt * 8 + tq * 2;
+        if (col >= valid) { s[nt][0] = -INFINITY; s[nt][2] = -INFINITY; }
+        if (col + 1 >= valid) { s[nt][1] = -INFINITY; s[nt][3] = -INFINITY; }
+      }
+      float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+      float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      const float n0 = fmaxf(m0, mx0 * sl2);
+      const float n1 = fmaxf(m1, mx1 * sl2);
+      const float u0 = (n0 == -INFINITY) ? 0.0f : n0;
+      const float u1 = (n1 == -INFINITY) ? 0.0f : n1;
+      const float a0 = ex2(m0 - u0);
+      const float a1 = ex2(m1 - u1);
+      m0 = n0;
+      m1 = n1;
+      float pr[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        pr[nt][0] = ex2(fmaf(s[nt][0], sl2, -u0));
+        pr[nt][1] = ex2(fmaf(s[nt][1], sl2, -u0));
+        pr[nt][2] = ex2(fmaf(s[nt][2], sl2, -u1));
+        pr[nt][3] = ex2(fmaf(s[nt][3], sl2, -u1));
+      }
+      l0 = l0 * a0 + pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1];
+      l1 = l1 * a1 + pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        o[j][0] *= a0;
+        o[j][1] *= a0;
+        o[j][2] *= a1;
+        o[j][3] *= a1;
+      }
+      uint32_t pa[4];
+      pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
+      pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
+      pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
+      pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+      // O += P V: 16 d-tiles of 8, two per transposed ldmatrix.x4
+      {
+        const int mi = lane >> 3, rr = lane & 7;
+        const int key = (mi & 1) * 8 + rr;
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(sv + swz(key, j + (mi >> 1)), b0, b1, b2, b3);
+          mma16816(o[j], pa, b0, b1);
+          mma16816(o[j + 1], pa, b2, b3);
+        }
+      }
+      __syncwarp();   // this slot is refilled only after every lane has read it
+    }
+    // partial of this piece: normalise and write rows < G
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    const float inv0 = (l0 > 0.0f) ? 1.0f / l0 : 0.0f;
+    const float inv1 = (l1 > 0.0f) ? 1.0f / l1 : 0.0f;
+    if (gr < p.group) {
+      float* dst = p.o_part + (prow + gr) * 128;
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        *reinterpret_cast<float2*>(dst + j * 8 + tq * 2) = make_float2(o[j][0] * inv0, o[j][1] * inv0);
+      if (tq == 0) p.lse_part[prow + gr] = (l0 > 0.0f) ? (m0 + log2f(l0)) * 0.69314718055994531f : -INFINITY;
+    }
+    if (gr + 8 < p.group) {
+      float* dst = p.o_part + (prow + gr + 8) * 128;
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        *reinterpret_cast<float2*>(dst + j * 8 + tq * 2) = make_float2(o[j][2] * inv1, o[j][3] * inv1);
+      if (tq == 0) p.lse_part[prow + gr + 8] = (l1 > 0.0f) ? (m1 + log2f(l1)) * 0.69314718055994531f : -INFINITY;
     }
   }
   cp_async_wait<0>();
-  __syncthreads();
-
-  // combine the four warps: rows gr and gr+8 of each warp
-  float* sm_o = reinterpret_cast<float*>(smem);                 // [4][16][128]
-  float* sm_m = sm_o + 4 * 16 * 128;                            // [4][16]
-  float* sm_l = sm_m + 4 * 16;                                  // [4][16]
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  if (tq == 0) {
-    sm_m[warp * 16 + gr] = m0;
-    sm_m[warp * 16 + gr + 8] = m1;
-    sm_l[warp * 16 + gr] = l0;
-    sm_l[warp * 16 + gr + 8] = l1;
-  }
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const int col = j * 8 + tq * 2;
-    sm_o[(warp * 16 + gr) * 128 + col] = o[j][0];
-    sm_o[(warp * 16 + gr) * 128 + col + 1] = o[j][1];
-    sm_o[(warp * 16 + gr + 8) * 128 + col] = o[j][2];
-    sm_o[(warp * 16 + gr + 8) * 128 + col + 1] = o[j][3];
-  }
-  __syncthreads();
-  {
-    const int row = threadIdx.x >> 3;  // 16 rows, 8 threads each, 16 columns per thread
-    const int c0 = (threadIdx.x & 7) * 16;
-    float mw[4], M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      mw[w] = sm_m[w * 16 + row];
-      M = fmaxf(M, mw[w]);
-    }
-    float L = 0.0f, sc[4];
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      sc[w] = (M == -INFINITY) ? 0.0f : ex2(mw[w] - M);
-      L += sm_l[w * 16 + row] * sc[w];
-    }
-    if (row < p.group) {
-      const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
-      const size_t prow = (static_cast<size_t>(split) * p.batch + b) * p.n_h + g * p.group + row;
-      float* dst = p.o_part + prow * 128 + c0;
-#pragma unroll
-      for (int i = 0; i < 16; i += 4) {
-        float4 acc;
-        acc.x = (sm_o[(0 * 16 + row) * 128 + c0 + i + 0] * sc[0] + sm_o[(1 * 16 + row) * 128 + c0 + i + 0] * sc[1] +
-                 sm_o[(2 * 16 + row) * 128 + c0 + i + 0] * sc[2] + sm_o[(3 * 16 + row) * 128 + c0 + i + 0] * sc[3]) * inv;
-        acc.y = (sm_o[(0 * 16 + row) * 128 + c0 + i + 1] * sc[0] + sm_o[(1 * 16 + row) * 128 + c0 + i + 1] * sc[1] +
-                 sm_o[(2 * 16 + row) * 128 + c0 + i + 1] * sc[2] + sm_o[(3 * 16 + row) * 128 + c0 + i + 1] * sc[3]) * inv;
-        acc.z = (sm_o[(0 * 16 + row) * 128 + c0 + i + 2] * sc[0] + sm_o[(1 * 16 + row) * 128 + c0 + i + 2] * sc[1] +
-                 sm_o[(2 * 16 + row) * 128 + c0 + i + 2] * sc[2] + sm_o[(3 * 16 + row) * 128 + c0 + i + 2] * sc[3]) * inv;
-        acc.w = (sm_o[(0 * 16 + row) * 128 + c0 + i + 3] * sc[0] + sm_o[(1 * 16 + row) * 128 + c0 + i + 3] * sc[1] +
-                 sm_o[(2 * 16 + row) * 128 + c0 + i + 3] * sc[2] + sm_o[(3 * 16 + row) * 128 + c0 + i + 3] * sc[3]) * inv;
-        *reinterpret_cast<float4*>(dst + i) = acc;
-      }
-      if ((threadIdx.x & 7) == 0)
-        p.lse_part[prow] = (L > 0.0f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
-    }
-  }
 }
 
-// Merge of the split partials of one (request, head) per CTA: the 8 warps take
-// every 8th split, each keeps an online (max, sum, O) over its splits with
-// float4 loads eight splits deep, and the eight results are combined in shared
-// memory. Same formula as the generic merge (LSE weighting, -inf splits weigh
-// 0); more warps per row so the 256 splits stream at full bandwidth.
+// Merge of the partials of one (request, head) per CTA. The pieces of pair bg
+// come from the warps whose ranges hold its first and last flattened keys and
+// every warp in between with a non-empty range; warp w's piece is in slot
+// w + bg. The 8 warps take every 8th piece, each keeps an online (max, sum, O)
+// with float4 loads four pieces deep, and the eight results are combined in
+// shared memory. Same formula as the generic merge (LSE weighting, -inf
+// partials weigh 0). This kernel also checks the offsets of its request and
+// records kStatusInternal for offsets that break the contract.
 constexpr int kMergeThreads = 256;
-constexpr int kMergeUnroll = 8;
+constexpr int kMergeUnroll = 4;
 
-__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const float* __restrict__ o_parts,
-                                                                      const float* __restrict__ lse_parts,
-                                                                      int n_splits, int64_t n_rowheads,
+__global__ void __launch_bounds__(kMergeThreads, 4) decode_merge_kernel(const __grid_constant__ Params p,
                                                                       __nv_bfloat16* out, float* lse_out) {
   __shared__ float sm_m[8], sm_l[8];
   __shared__ float4 sm_o[8][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t rh = blockIdx.x;
-  const int64_t o_stride = n_rowheads * 128;   // floats between splits
+  const int b = static_cast<int>(rh / p.n_h);
+  const int h = static_cast<int>(rh - static_cast<int64_t>(b) * p.n_h);
+  const int g = h / p.group;
+  const int hl = h - g * p.group;
+  const int bg = b * p.n_kv + g;
+  const int64_t o0 = p.offsets[0], oB = p.offsets[p.batch];
+  const int64_t base = p.offsets[b], end = p.offsets[b + 1];
+  const bool ok = o0 >= 0 && oB >= o0 && oB <= p.kv_rows && base >= o0 && end >= base && end <= oB;
+  if (!ok && threadIdx.x == 0) atomicOr(p.status, kStatusInternal);
+  const int64_t len = ok ? end - base : 0;
+  const int64_t kt = (oB - o0) * p.n_kv;
+  const int64_t W = p.n_warps;
+  int64_t w_first = 0, n_pieces = 0;
+  if (len > 0) {
+    const int64_t vs = (base - o0) * p.n_kv + g * len;
+    w_first = range_of(vs, kt, W);
+    n_pieces = range_of(vs + len - 1, kt, W) - w_first + 1;
+  }
   float m = -INFINITY, l = 0.0f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j0 = warp; j0 < n_splits; j0 += 8 * kMergeUnroll) {
+  for (int64_t j0 = warp; j0 < n_pieces; j0 += 8 * kMergeUnroll) {
+    // pieces present (a range is empty only when there are fewer keys than ranges)
+    uint32_t present = 0;
+#pragma unroll 1
+    for (int u = 0; u < kMergeUnroll; ++u) {
+      const int64_t w = w_first + j0 + u * 8;
+      if (j0 + u * 8 < n_pieces && (kt >= W || range_start(w, kt, W) < range_start(w + 1, kt, W)))
+        present |= 1u << u;
+    }
     float4 x[kMergeUnroll];
     float lj[kMergeUnroll];
 #pragma unroll
     for (int u = 0; u < kMergeUnroll; ++u) {
-      const int j = j0 + u * 8;
       lj[u] = -INFINITY;
       x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j < n_splits) {
-        lj[u] = __ldg(lse_parts + j * n_rowheads + rh);
-        x[u] = __ldcs(reinterpret_cast<const float4*>(o_parts + j * o_stride + rh * 128) + lane);
+      if (present & (1u << u)) {
+        const int64_t row = (w_first + j0 + u * 8 + bg) * p.group + hl;
+        lj[u] = __ldcs(p.lse_part + row);
+        x[u] = __ldcs(reinterpret_cast<const float4*>(p.o_part + row * 128) + lane);
       }
     }
 #pragma unroll
@@ -351,7 +440,7 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const float
     if (M != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < 8; ++w) {
-        const float sc = expf(sm_m[w] - M);   // 0 for warps that saw no split
+        const float sc = expf(sm_m[w] - M);   // 0 for warps that saw no piece
         L += sm_l[w] * sc;
         const float4 a = sm_o[w][lane];
         o.x = fmaf(sc, a.x, o.x);

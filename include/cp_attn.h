@@ -161,8 +161,9 @@ cp_status cp_ring_comm_volume(const cp_range* ranges, const cp_block* blocks, in
 
 /* Bytes of workspace an entry point needs (always a multiple of 256).
  *  CP_OP_PARTIAL, CP_OP_MERGE: 256 (the status word).
- *  CP_OP_DECODE: 256 + the split partials, n_splits*batch*n_h*(d+1)*4 rounded
- *  up to 256. `rows` is the batch for decode. */
+ *  CP_OP_DECODE: 256 + room for ((n_splits+1)*batch + 7)*n_h partial rows of
+ *  d+1 floats (O and LSE), each part rounded up to 256; a bound on what
+ *  cp_decode uses on any device. `rows` is the batch for decode. */
 size_t cp_workspace_size(cp_op op, int64_t rows, int32_t n_h, int32_t d, int32_t n_splits);
 
 /* Zero the status word of a workspace (stream-ordered). */
@@ -215,16 +216,25 @@ cp_status cp_attn_merge(const float* o_parts, const float* lse_parts, int32_t n_
                         int64_t part_stride_rows, int64_t rows, int32_t n_h, int32_t d, void* out,
                         cp_dtype out_dtype, float* lse_out, void* cuda_stream);
 
-/* Split-KV decode (Flash Decoding with n_splits splits per request; method
- * page, section 5 software stack). Request b has one query row q[b] at
- * position L_b - 1 and keys k/v rows kv_offsets[b] .. kv_offsets[b+1]-1
- * (L_b = difference), all visible. Split s covers request keys
- * [floor(s*L_b/n_splits), floor((s+1)*L_b/n_splits)); each split's partial
- * goes to the workspace, then the splits are merged as in cp_attn_merge.
+/* Split-KV decode (Flash Decoding; method page, section 5 software stack).
+ * Request b has one query row q[b] at position L_b - 1 and keys k/v rows
+ * kv_offsets[b] .. kv_offsets[b+1]-1 (L_b = difference), all visible.
+ * The splits are cut over the whole batch rather than per request: the keys
+ * of every (request, KV head) pair, in order, form one sequence of
+ * Kt = n_kv*(kv_offsets[batch] - kv_offsets[0]) keys, cut into W equal ranges,
+ * W = 8*min(SM count, ceil(n_splits*batch*n_kv/8)). So n_splits caps the
+ * average number of splits per pair, and every range holds the same number
+ * of keys whatever the mix of lengths. Each range leaves one partial per pair
+ * it overlaps in the workspace; the partials of each (request, head) are then
+ * merged as in cp_attn_merge. The result does not depend on the cut beyond
+ * rounding.
  *   q [batch, n_h, d] bf16; k, v [kv_rows, n_kv, d] bf16;
- *   kv_offsets: DEVICE int64 [batch+1], non-decreasing, last <= kv_rows;
+ *   kv_offsets: DEVICE int64 [batch+1], non-decreasing, last <= kv_rows
+ *   (with offsets that break this no K/V row outside [0, kv_rows) is read,
+ *   and cp_check_status then reports CP_ERR_INTERNAL);
  *   out [batch, n_h, d] bf16; lse_out [batch, n_h] fp32 (may be NULL).
- * Supports dtype CP_BF16, d == 128, n_h/n_kv == 16, 1 <= n_splits <= 1024.
+ * Supports dtype CP_BF16, d == 128, n_h/n_kv in {1, 2, 4, 8, 16},
+ * 1 <= n_splits <= 1024, Kt*W < 2^53.
  * A request with L_b = 0 yields out = 0, lse = -inf.
  * workspace: >= cp_workspace_size(CP_OP_DECODE, batch, n_h, d, n_splits). */
 cp_status cp_decode(const void* q, const void* k, const void* v, cp_dtype dtype,
@@ -240,8 +250,9 @@ cp_status cp_decode(const void* q, const void* k, const void* v, cp_dtype dtype,
  * Same arguments, results and limits as cp_decode, without the workspace: the
  * split partials live in a fixed 32 MiB array in the library's device memory,
  * which every GPU that loads the library holds until the process exits.
- *  - Requests whose cp_workspace_size(CP_OP_DECODE, batch, n_h, d, n_splits)
- *    exceeds 32 MiB are rejected with CP_ERR_WORKSPACE before any launch.
+ *  - Requests whose partials, (W + batch*n_kv)*(n_h/n_kv) rows of d+1 floats
+ *    with W as in cp_decode for the current device, need more than the array
+ *    are rejected with CP_ERR_WORKSPACE before any launch.
  *  - The first call on a device looks up the array's device address for that
  *    device (the device current at the call); make that first call before any
  *    stream capture.

@@ -193,3 +193,19 @@ def test_decode(n_h, n_kv, n_splits):
     B.cp_check_status(ws)
     o_ref, l_ref = OD.decode(dc.q, dc.k, dc.v, dc.offsets)
     check(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "bf16", "decode")
+
+
+def test_decode_reports_decreasing_offsets():
+    """Offsets that decrease are reported through the status word; every row
+    read stays inside the K/V rows the call was given."""
+    lens = [100, 60, 140]
+    dc = synth.make_decode(len(lens), 16, 1, 128, lens, 77, 0.5)
+    q, k, v = dev(dc.q_raw, "bf16"), dev(dc.k_raw, "bf16"), dev(dc.v_raw, "bf16")
+    bad = torch.tensor([0, 100, 50, 300], dtype=torch.int64, device="cuda")   # request 1 ends before it starts
+    out = torch.empty((3, 16, 128), dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(B.cp_workspace_size(B.CP_OP_DECODE, 3, 16, 128, 16), dtype=torch.uint8, device="cuda")
+    B.cp_decode(q, k, v, bad, 16, 1, 16, 1 / math.sqrt(128), out, None, ws)
+    torch.cuda.synchronize()
+    with pytest.raises(B.CpError) as e:
+        B.cp_check_status(ws)
+    assert e.value.code == B.CP_ERR_INTERNAL

@@ -79,10 +79,10 @@ def test_rejects_requests_beyond_the_scratch_limit():
     q, k, v, off, n_h, n_kv = _case(73, [64, 64])
     out = torch.empty((2, n_h, 128), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((2, n_h), dtype=torch.float32, device="cuda")
-    # 1024 splits x 2 requests x 16 heads fit; 1024 splits x 600 requests do not (needs > 32 MiB)
-    big_q = torch.zeros((600, n_h, 128), dtype=torch.bfloat16, device="cuda")
-    big_off = torch.zeros(601, dtype=torch.int64, device="cuda")
-    big_out = torch.empty((600, n_h, 128), dtype=torch.bfloat16, device="cuda")
+    # 2 requests fit; 5000 requests do not: (8 x 148 ranges + 5000 pairs) x 16 heads x 129 floats > 32 MiB
+    big_q = torch.zeros((5000, n_h, 128), dtype=torch.bfloat16, device="cuda")
+    big_off = torch.zeros(5001, dtype=torch.int64, device="cuda")
+    big_out = torch.empty((5000, n_h, 128), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(B.CpError) as e:
         B.cp_decode_static(big_q, k, v, big_off, n_h, n_kv, 1024, 0.1, big_out, None)
     assert e.value.code == B.CP_ERR_WORKSPACE
