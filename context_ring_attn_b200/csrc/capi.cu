@@ -363,18 +363,30 @@ cp_status cp_attn_merge(const float* o_parts, const float* lse_parts, int32_t n_
   }
   const int64_t n_rowheads = rows * n_h;
   if (n_rowheads == 0) return CP_OK;
-  const int64_t warps_per_block = merge::kThreads / 32;
-  int64_t grid = (n_rowheads + warps_per_block - 1) / warps_per_block;
-  grid = std::min<int64_t>(grid, 148 * 32);
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   const int64_t o_stride = part_stride_rows * n_h * d;
   const int64_t l_stride = part_stride_rows * n_h;
-  if (out_dtype == CP_F32)
-    merge::merge_kernel<float><<<static_cast<unsigned>(grid), merge::kThreads, 0, stream>>>(
-        o_parts, lse_parts, n_parts, o_stride, l_stride, n_rowheads, d, static_cast<float*>(out), lse_out);
-  else
-    merge::merge_kernel<__nv_bfloat16><<<static_cast<unsigned>(grid), merge::kThreads, 0, stream>>>(
-        o_parts, lse_parts, n_parts, o_stride, l_stride, n_rowheads, d, static_cast<__nv_bfloat16*>(out), lse_out);
+  // (row, head) pairs per warp and round: 8 float4 loads per lane split over the parts
+  const int c = n_parts > 4 ? 8 : n_parts > 2 ? 4 : 2;
+  const int r = 8 / c;
+  const int64_t warps_per_block = merge::kThreads / 32;
+  int64_t grid = (n_rowheads + warps_per_block * r - 1) / (warps_per_block * r);
+  grid = std::min<int64_t>(grid, 148 * 32);
+  const unsigned g = static_cast<unsigned>(grid);
+  const unsigned t = merge::kThreads;
+#define CP_MERGE_LAUNCH(OutT, R_)                                                                          \
+  merge::merge_kernel<OutT, R_><<<g, t, 0, stream>>>(o_parts, lse_parts, n_parts, o_stride, l_stride, n_rowheads, d, \
+                                                     static_cast<OutT*>(out), lse_out)
+  if (out_dtype == CP_F32) {
+    if (r == 1) CP_MERGE_LAUNCH(float, 1);
+    else if (r == 2) CP_MERGE_LAUNCH(float, 2);
+    else CP_MERGE_LAUNCH(float, 4);
+  } else {
+    if (r == 1) CP_MERGE_LAUNCH(__nv_bfloat16, 1);
+    else if (r == 2) CP_MERGE_LAUNCH(__nv_bfloat16, 2);
+    else CP_MERGE_LAUNCH(__nv_bfloat16, 4);
+  }
+#undef CP_MERGE_LAUNCH
   return last_cuda_status();
 }
 

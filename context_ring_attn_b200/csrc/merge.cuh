@@ -5,9 +5,17 @@
 // out = sum_j exp(lse_j - lse) * o_j; parts at -inf weigh 0.
 //
 // HBM-bound: every partial is read once with 16-byte loads and the output is
-// written once. One warp per (row, head); lane l owns float4 columns
-// l, l+32, ...; the part weights are computed 32 parts at a time, one per lane,
-// and broadcast with shuffles while eight parts' loads are in flight.
+// written once. The weights are folded in online, eight partial rows per lane
+// per round: a warp takes R (row, head) pairs at a time and C = 8 / R parts of
+// each per round, loads their C LSEs (broadcast) together with the C float4s
+// of each row, then rescales its running (max, sum, O) once per round. So a
+// round costs one memory latency whatever n_parts is (R = 1, C = 8 for the
+// 8-way merge; R = 4, C = 2 for the running 2-way merge and for a single
+// part), and lane l owns the float4 columns l, l+32, ... of the rows.
+//
+// out may alias o_parts (part 0) and lse_out may alias lse_parts (part 0):
+// each lane reads all parts of its columns before writing them, and the LSE
+// is written after the warp has read every LSE it needs.
 #pragma once
 
 #include "common.cuh"
@@ -16,7 +24,7 @@ namespace cpk {
 namespace merge {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 8;
+constexpr int kLoads = 8;   // float4 loads per lane per round
 
 __device__ __forceinline__ void store4(float* dst, float4 v) { *reinterpret_cast<float4*>(dst) = v; }
 
@@ -27,66 +35,87 @@ __device__ __forceinline__ void store4(__nv_bfloat16* dst, float4 v) {
   *reinterpret_cast<uint2*>(dst) = u;
 }
 
-template <typename OutT>
-__global__ void __launch_bounds__(kThreads) merge_kernel(const float* __restrict__ o_parts,
+template <typename OutT, int R>
+__global__ void __launch_bounds__(kThreads, R <= 2 ? 3 : 2) merge_kernel(const float* __restrict__ o_parts,
                                                           const float* __restrict__ lse_parts, int n_parts,
                                                           int64_t o_stride, int64_t l_stride, int64_t n_rowheads,
                                                           int d, OutT* out, float* lse_out) {
+  constexpr int C = kLoads / R;
   const int lane = threadIdx.x & 31;
   const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
   const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
   const int n_vec = d >> 2;
 
-  for (int64_t rh = warp_global; rh < n_rowheads; rh += n_warps) {
-    // pass 1: max and sum of the part LSEs
-    float mx = -INFINITY;
-    for (int j = lane; j < n_parts; j += 32) mx = fmaxf(mx, lse_parts[j * l_stride + rh]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float lse;
-    if (mx == -INFINITY) {
-      lse = -INFINITY;
-    } else {
-      float sum = 0.0f;
-      for (int j = lane; j < n_parts; j += 32) sum += expf(lse_parts[j * l_stride + rh] - mx);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      lse = mx + logf(sum);
-    }
-    // pass 2: weighted sum of the part outputs
+  for (int64_t rh0 = warp_global * R; rh0 < n_rowheads; rh0 += n_warps * R) {
+    float lse_r[R];
     for (int vbase = 0; vbase < n_vec; vbase += 32) {
       const int vi = vbase + lane;
       const bool active = vi < n_vec;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (lse != -INFINITY) {
-        for (int jb = 0; jb < n_parts; jb += 32) {
-          const int jl = jb + lane;
-          const float w_lane = (jl < n_parts) ? expf(lse_parts[jl * l_stride + rh] - lse) : 0.0f;
-          const int cnt = min(32, n_parts - jb);
-          for (int jj = 0; jj < cnt; jj += kUnroll) {
-            float4 x[kUnroll];
+      float m[R], l[R];
+      float4 acc[R];
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-              x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-              if (active && jj + u < cnt)
-                x[u] = __ldcs(reinterpret_cast<const float4*>(o_parts + (jb + jj + u) * o_stride + rh * d) + vi);
-            }
+      for (int r = 0; r < R; ++r) {
+        m[r] = -INFINITY;
+        l[r] = 0.0f;
+        acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      for (int jb = 0; jb < n_parts; jb += C) {
+        float lj[R][C];
+        float4 x[R][C];
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-              const float w = __shfl_sync(0xffffffffu, w_lane, (jj + u) & 31);
-              if (jj + u < cnt && w != 0.0f) {
-                acc.x = fmaf(w, x[u].x, acc.x);
-                acc.y = fmaf(w, x[u].y, acc.y);
-                acc.z = fmaf(w, x[u].z, acc.z);
-                acc.w = fmaf(w, x[u].w, acc.w);
-              }
+        for (int r = 0; r < R; ++r) {
+#pragma unroll
+          for (int c = 0; c < C; ++c) {
+            const int64_t rh = rh0 + r;
+            const int j = jb + c;
+            lj[r][c] = -INFINITY;
+            x[r][c] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (rh < n_rowheads && j < n_parts) {
+              lj[r][c] = lse_parts[j * l_stride + rh];
+              if (active) x[r][c] = __ldcs(reinterpret_cast<const float4*>(o_parts + j * o_stride + rh * d) + vi);
             }
           }
         }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          float mx = lj[r][0];
+#pragma unroll
+          for (int c = 1; c < C; ++c) mx = fmaxf(mx, lj[r][c]);
+          const float m_new = fmaxf(m[r], mx);
+          const float mu = (m_new == -INFINITY) ? 0.0f : m_new;   // parts at -inf weigh 0
+          const float sc = expf(m[r] - mu);
+          l[r] *= sc;
+          acc[r].x *= sc;
+          acc[r].y *= sc;
+          acc[r].z *= sc;
+          acc[r].w *= sc;
+#pragma unroll
+          for (int c = 0; c < C; ++c) {
+            const float w = expf(lj[r][c] - mu);
+            l[r] += w;
+            acc[r].x = fmaf(w, x[r][c].x, acc[r].x);
+            acc[r].y = fmaf(w, x[r][c].y, acc[r].y);
+            acc[r].z = fmaf(w, x[r][c].z, acc[r].z);
+            acc[r].w = fmaf(w, x[r][c].w, acc[r].w);
+          }
+          m[r] = m_new;
+        }
       }
-      if (active) store4(out + rh * d + vi * 4, acc);
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int64_t rh = rh0 + r;
+        const float inv = (l[r] > 0.0f) ? 1.0f / l[r] : 0.0f;
+        lse_r[r] = (l[r] > 0.0f) ? m[r] + logf(l[r]) : -INFINITY;
+        if (rh < n_rowheads && active)
+          store4(out + rh * d + vi * 4, make_float4(acc[r].x * inv, acc[r].y * inv, acc[r].z * inv, acc[r].w * inv));
+      }
     }
-    if (lse_out && lane == 0) lse_out[rh] = lse;
+    __syncwarp();   // every lane has read the LSEs before part 0's may be overwritten
+    if (lse_out && lane == 0) {
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+        if (rh0 + r < n_rowheads) lse_out[rh0 + r] = lse_r[r];
+    }
   }
 }
 

@@ -148,11 +148,14 @@ def test_bf16_partial_empty_rows():
 
 
 # ---------------------------------------------------------------------------- merge
-@pytest.mark.parametrize("n_parts,d,out_dtype", [(1, 128, "f32"), (3, 64, "f32"), (8, 128, "bf16"),
-                                                 (40, 128, "f32"), (256, 128, "bf16")])
-def test_merge(n_parts, d, out_dtype):
+@pytest.mark.parametrize("n_parts,d,out_dtype,n_h", [(1, 128, "f32", 4), (3, 64, "f32", 4), (8, 128, "bf16", 4),
+                                                      (40, 128, "f32", 4), (256, 128, "bf16", 4),
+                                                      (2, 128, "f32", 3), (5, 128, "bf16", 3), (3, 128, "f32", 3)])
+def test_merge(n_parts, d, out_dtype, n_h):
+    """Part counts that take every grouping of (row, head) pairs per warp and
+    parts per round, with row-head counts (148, 111) that leave ragged tails."""
     rng = np.random.default_rng(n_parts)
-    rows, n_h = 37, 4
+    rows = 37
     o = rng.standard_normal((n_parts, rows, n_h, d)).astype(np.float32)
     lse = (rng.standard_normal((n_parts, rows, n_h)) * 3).astype(np.float32)
     lse[rng.random(lse.shape) < 0.2] = -np.inf
