@@ -11,18 +11,25 @@
 // One CTA = two 128-row query tiles (a, b) of one KV head. GQA packing: each
 // tile's rows are (token, head-in-group) pairs, 128/G tokens x G query heads
 // that share the KV head (section 8.2 of the GQA page), so every K/V tile is
-// loaded once for 2 x 128 rows. Warp roles (320 threads):
-//   warps 0-3  softmax of tile a, warps 4-7 softmax of tile b: thread = row.
-//              It reads its S row from TMEM, masks by global position, keeps
-//              the running max, writes P (bf16 pairs) over its own S row in
-//              TMEM, rescales its O row in TMEM when the running max grows by
-//              more than 2^8, and writes the normalised O row and its LSE;
-//   warp 8     TMA producers: lane 0 loads Q, then K tiles into a 3-stage
+// loaded once for 2 x 128 rows. Warp roles (576 threads):
+//   warps 0-7  softmax of tile a, warps 8-15 softmax of tile b. Two threads
+//              per row: warps w and w+4 read the same TMEM lane quarter, one
+//              the 64 columns 0-63 of the row, the other 64-127. Per KV tile
+//              each reads its half of the S row from TMEM, masks by global
+//              position, exchanges its half-row max with its partner through
+//              shared memory (a 64-thread named barrier), writes its P half
+//              (bf16 pairs) over the S row in TMEM, keeps its own part of the
+//              row sum, and rescales its half of the O row when the running
+//              max grows by more than 2^8; at the end the two sums are added
+//              and each thread writes half of the normalised O row;
+//   warp 16    TMA producers: lane 0 loads Q, then K tiles into a 3-stage
 //              ring; lane 1 loads V tiles into a 2-stage ring;
-//   warp 9     MMA issuer (one thread) and TMEM owner. Per KV tile j it issues
+//   warp 17    MMA issuer (one thread) and TMEM owner. Per KV tile j it issues
 //              O_a += P_a(j) V_j, S_a(j+1) = Q_a K_{j+1}^T, O_b += P_b(j) V_j,
 //              S_b(j+1) = Q_b K_{j+1}^T, so that one tile's softmax always
 //              overlaps the other tile's MMAs (ping-pong).
+// Two threads per row halve the latency of a softmax step, which otherwise
+// exceeds the MMA time of one tile and stalls the ping-pong.
 // TMEM (512 columns): S_a 0, S_b 128 (P over the first 64 columns), O_a 256,
 // O_b 384. tcgen05 operations of one thread complete in issue order, so the
 // completion of S_x(j+1) also means O_x += P_x(j) V_j has completed.
@@ -42,17 +49,18 @@ constexpr int kHalfBytes = 128 * 128;        // 128 rows x 64 bf16 (one 128-byte
 constexpr int kTileBytes = 2 * kHalfBytes;   // 128 rows x 128 bf16
 constexpr int kKStages = 3;
 constexpr int kVStages = 2;
-constexpr int kSoftmaxWarps = 8;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kThreads = 320;
+constexpr int kSoftmaxWarps = 16;
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kThreads = 576;
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kQTiles * kTileBytes;
 constexpr int kOffV = kOffK + kKStages * kTileBytes;
 constexpr int kOffBar = kOffV + kVStages * kTileBytes;
 constexpr int kNumBars = 24;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kSmemNeeded = kOffMisc + 16;
+constexpr int kOffXch = kOffMisc + 16;                 // [tile][half][row] f32: half-row max, then sum
+constexpr int kSmemNeeded = kOffXch + kQTiles * 2 * BM * 4;
 constexpr int kSmemMax = 232448;                     // 227 KB per block on sm_100
 // The dynamic shared window starts 1024-aligned in practice; whatever slack is
 // left covers a smaller alignment, and the kernel checks it at run time.
@@ -72,7 +80,7 @@ enum {
   B_V_FULL = 7,     // +stage (2)
   B_V_EMPTY = 9,    // +stage (2)
   B_S_FULL = 11,    // +tile: S_x(j) is in TMEM (and O_x += P_x(j-1) V is done)
-  B_P_FULL = 13,    // +tile (4 arrivals): P_x(j) is in TMEM
+  B_P_FULL = 13,    // +tile (8 arrivals): P_x(j) is in TMEM
   B_O_DONE = 15,    // +tile: O_x += P_x(j) V_j has completed
   B_DRAIN = 17
 };
@@ -110,7 +118,9 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint3
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1) partial_bf16_kernel(const __grid_constant__ Params p) {
+// 18 warps put five on two of the four schedulers, whose register files hold
+// 16K registers each: at most 102 per thread, so 96.
+__global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
@@ -148,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1) partial_bf16_kernel(const __grid_
   }
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNumBars; ++i) mbar_init(&bars[i], (i == B_P_FULL || i == B_P_FULL + 1) ? 4u : 1u);
+    for (int i = 0; i < kNumBars; ++i) mbar_init(&bars[i], (i == B_P_FULL || i == B_P_FULL + 1) ? 8u : 1u);
     *abort_flag = 0u;
     fence_mbar_init();
   }
@@ -264,19 +274,24 @@ __global__ void __launch_bounds__(kThreads, 1) partial_bf16_kernel(const __grid_
       drain_wait(&bars[B_DRAIN], 0u, p.status);
     }
   } else {
-    // ------------------------------------------------------------------ softmax warps 0..7
-    const int x = warp >> 2;                // query tile of this warpgroup
+    // ------------------------------------------------------------------ softmax warps 0..15
+    const int x = warp >> 3;                // query tile of this warp
+    const int hf = (warp >> 2) & 1;         // half of the row: columns hf*64 .. hf*64+63
     const int quarter = warp & 3;           // TMEM lane quarter
     const int row = quarter * 32 + lane;    // packed row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t s_col = tmem + lane_base + kColS + x * BN;
-    const uint32_t o_col = tmem + lane_base + kColO + x * HD;
+    const uint32_t s_col = tmem + lane_base + kColS + x * BN + hf * 64;   // this thread's S columns
+    const uint32_t p_col = tmem + lane_base + kColS + x * BN + hf * 32;   // its P columns (bf16 pairs)
+    const uint32_t o_col = tmem + lane_base + kColO + x * HD + hf * 64;   // its O columns
+    float* xch_mine = reinterpret_cast<float*>(smem + kOffXch) + (x * 2 + hf) * BM + row;
+    const float* xch_peer = reinterpret_cast<const float*>(smem + kOffXch) + (x * 2 + (hf ^ 1)) * BM + row;
+    const uint32_t pair_bar = 1 + x * 4 + quarter;   // named barrier of the two warps sharing these rows
     const int tok = x * tok_per_tile + (row >> p.log2_group);   // token within the CTA
     const bool row_valid = tok < n_tok;
     const int64_t qpos = q_pos_lo + tok;
     const float sl2 = p.scale_log2;
     float m_run = -INFINITY;
-    float l_run = 0.0f;
+    float l_run = 0.0f;   // this thread's part of the row sum
     bool ok = true;
     int it = 0;
 
@@ -288,32 +303,30 @@ __global__ void __launch_bounds__(kThreads, 1) partial_bf16_kernel(const __grid_
         const int64_t kp0 = kr.pos0 + k0;
         const int n_valid = static_cast<int>(min(static_cast<int64_t>(BN), nv - k0));
         // S_x(it) is in TMEM; this also means O_x += P_x(it-1) V has completed
-        if (!warp_wait(&bars[B_S_FULL + x], it & 1, abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
-        uint32_t s[4][32];
+        const bool got = warp_wait(&bars[B_S_FULL + x], it & 1, abort_flag, p.status);
+        uint32_t s[2][32];
+        float mx = -INFINITY;
+        // key hf*64 + c of the tile is visible iff c <= lim
+        int lim = 63;
+        if (got) {
+          tc_fence_after();
+          tmem_ld32(s_col, s[0]);
+          tmem_ld32(s_col + 32, s[1]);
+          tmem_ld_wait();
+          if ((n_valid < BN) || (causal && kp0 + BN - 1 > qpos)) {
+            int64_t l64 = n_valid - 1;
+            if (causal && qpos - kp0 < l64) l64 = qpos - kp0;
+            l64 -= hf * 64;
+            lim = static_cast<int>(max(min(l64, static_cast<int64_t>(63)), static_cast<int64_t>(-1)));
+          }
+          if (__any_sync(0xffffffffu, lim < 63)) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(s_col + c * 32, s[c]);
-        tmem_ld_wait();
-
-        // key c of the tile is visible iff c <= lim
-        int lim = BN - 1;
-        if ((n_valid < BN) || (causal && kp0 + BN - 1 > qpos)) {
-          int64_t l64 = n_valid - 1;
-          if (causal && qpos - kp0 < l64) l64 = qpos - kp0;
-          lim = static_cast<int>(max(l64, static_cast<int64_t>(-1)));
-        }
-        const bool masked = __any_sync(0xffffffffu, lim < BN - 1);
-        if (masked) {
-#pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (c > lim) s[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-        }
-        // row max: four chains of 3-input max
-        float mx;
-        {
+            for (int c = 0; c < 64; ++c)
+              if (c > lim) s[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+          }
           float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < BN; c += 8) {
+          for (int c = 0; c < 64; c += 8) {
             a0 = fmax3(a0, __uint_as_float(s[c >> 5][(c + 0) & 31]), __uint_as_float(s[c >> 5][(c + 1) & 31]));
             a1 = fmax3(a1, __uint_as_float(s[c >> 5][(c + 2) & 31]), __uint_as_float(s[c >> 5][(c + 3) & 31]));
             a2 = fmax3(a2, __uint_as_float(s[c >> 5][(c + 4) & 31]), __uint_as_float(s[c >> 5][(c + 5) & 31]));
@@ -321,6 +334,19 @@ __global__ void __launch_bounds__(kThreads, 1) partial_bf16_kernel(const __grid_
           }
           mx = fmaxf(fmax3(a0, a1, a2), a3);
         }
+        // Row max across the two halves. Both warps always meet here once per
+        // KV tile and agree on whether to go on, so neither can wait alone.
+        // The peer reads this slot before it arrives on P_FULL, and the next
+        // write comes after S_FULL, which needs that arrival: no overwrite race.
+        // The barrier also orders the partner's completed S loads before this
+        // thread's P stores, which overwrite S columns 32-63 (the tcgen05
+        // fences carry that order across the thread sync).
+        *xch_mine = mx;
+        tc_fence_before();
+        if (!named_bar_and(pair_bar, 64, got)) { ok = false; break; }
+        tc_fence_after();
+        mx = fmaxf(mx, *xch_peer);
+
         const float m_new = fmaxf(m_run, mx * sl2);
         float alpha = 1.0f;
         bool resc = false;
@@ -332,56 +358,60 @@ __global__ void __launch_bounds__(kThreads, 1) partial_bf16_kernel(const __grid_
         const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
         // p = 2^(s * scale * log2 e - m) in packed pairs: kPolyPairsPer8 of every
         // 8 pairs through the polynomial on the FMA pipe, the rest through the
-        // special-function unit. P goes back over the S row as bf16 pairs, 32
-        // columns at a time; the row sum runs in four packed chains.
+        // special-function unit. P goes back over the S row as bf16 pairs, 8
+        // columns (16 keys) at a time; the row sum runs in two packed chains.
         const uint64_t sl2_2 = f2_pack(sl2, sl2);
         const uint64_t negm_2 = f2_pack(-m_use, -m_use);
-        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+        uint64_t acc[2] = {0ull, 0ull};
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t pk[16];
+        for (int h8 = 0; h8 < 4; ++h8) {
+          uint32_t pk[8];
 #pragma unroll
-          for (int cc = 0; cc < 32; cc += 2) {
-            const int c = q4 * 32 + cc;
-            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[q4][cc]), __uint_as_float(s[q4][cc + 1])), sl2_2, negm_2);
+          for (int cc = 0; cc < 16; cc += 2) {
+            const int c = h8 * 16 + cc;
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[c >> 5][c & 31]), __uint_as_float(s[c >> 5][(c + 1) & 31])),
+                                       sl2_2, negm_2);
             uint64_t p2;
             if (((c >> 1) & 7) < kPolyPairsPer8) {
               p2 = exp2_poly_x2(x2);
+              // hidden keys contribute exactly zero (the polynomial leaves a tiny value there)
+              if (lim < 63) {
+                float p0, p1;
+                f2_unpack(p2, p0, p1);
+                if (c > lim) p0 = 0.0f;
+                if (c + 1 > lim) p1 = 0.0f;
+                p2 = f2_pack(p0, p1);
+              }
             } else {
               float x0, x1;
               f2_unpack(x2, x0, x1);
-              p2 = f2_pack(ex2(x0), ex2(x1));
+              p2 = f2_pack(ex2(x0), ex2(x1));   // ex2(-inf) is exactly 0
             }
             float p0, p1;
             f2_unpack(p2, p0, p1);
-            if (masked) {   // hidden keys contribute exactly zero (the polynomial leaves a tiny value)
-              if (c > lim) p0 = 0.0f;
-              if (c + 1 > lim) p1 = 0.0f;
-              p2 = f2_pack(p0, p1);
-            }
             pk[cc >> 1] = pack_bf16x2(p0, p1);
-            acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], p2);
+            acc[(c >> 1) & 1] = f2_add(acc[(c >> 1) & 1], p2);
           }
-          tmem_st16(s_col + q4 * 16, pk);
+          tmem_st8(p_col + h8 * 8, pk);
         }
         float sum;
         {
-          const uint64_t t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+          const uint64_t t = f2_add(acc[0], acc[1]);
           float lo, hi;
           f2_unpack(t, lo, hi);
           sum = lo + hi;
         }
         l_run = l_run * alpha + sum;
-        // O_x holds every earlier PV (see S_FULL above): rescale it in place if needed
+        // O_x holds every earlier PV (see S_FULL above): rescale this half in place if needed
         if (it > 0 && __any_sync(0xffffffffu, resc)) {
-#pragma unroll
+#pragma unroll 1
           for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(o_col + c * 32, o);
+            uint32_t o[16];
+            tmem_ld16(o_col + c * 16, o);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(o_col + c * 32, o);
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st16(o_col + c * 16, o);
           }
         }
         tmem_st_wait();
@@ -395,34 +425,36 @@ __global__ void __launch_bounds__(kThreads, 1) partial_bf16_kernel(const __grid_
     const int64_t out_row = ws.out_row0 + q_row0 + tok;
     const int head = kvh * group + (row & (group - 1));
     bool done_ok = __all_sync(0xffffffffu, ok);
+    if (done_ok && n_iter > 0) done_ok = warp_wait(&bars[B_O_DONE + x], (n_iter - 1) & 1, abort_flag, p.status);
+    // Whole row sum from the two halves. The partner warps agree on the
+    // outcome here as in the loop (both reach this barrier exactly once).
+    *xch_mine = l_run;
+    done_ok = named_bar_and(pair_bar, 64, done_ok);
+    const float l_tot = l_run + *xch_peer;
+    float* dst = p.o_part + (out_row * p.n_h + head) * HD + hf * 64;
     if (done_ok && n_iter > 0) {
-      done_ok = warp_wait(&bars[B_O_DONE + x], (n_iter - 1) & 1, abort_flag, p.status);
-      if (done_ok) {
-        tc_fence_after();
-        const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
-        float* dst = p.o_part + (out_row * p.n_h + head) * HD;
+      tc_fence_after();
+      const float inv_l = (l_tot > 0.0f) ? 1.0f / l_tot : 0.0f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld32(o_col + c * 32, o);
-          tmem_ld_wait();
-          if (row_valid) {
+      for (int c = 0; c < 2; ++c) {
+        uint32_t o[32];
+        tmem_ld32(o_col + c * 32, o);
+        tmem_ld_wait();
+        if (row_valid) {
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              float4 v4 = make_float4(__uint_as_float(o[i]) * inv_l, __uint_as_float(o[i + 1]) * inv_l,
-                                      __uint_as_float(o[i + 2]) * inv_l, __uint_as_float(o[i + 3]) * inv_l);
-              *reinterpret_cast<float4*>(dst + c * 32 + i) = v4;
-            }
+          for (int i = 0; i < 32; i += 4) {
+            float4 v4 = make_float4(__uint_as_float(o[i]) * inv_l, __uint_as_float(o[i + 1]) * inv_l,
+                                    __uint_as_float(o[i + 2]) * inv_l, __uint_as_float(o[i + 3]) * inv_l);
+            *reinterpret_cast<float4*>(dst + c * 32 + i) = v4;
           }
         }
       }
     } else if (done_ok && n_iter == 0 && row_valid) {
-      float* dst = p.o_part + (out_row * p.n_h + head) * HD;
 #pragma unroll
-      for (int i = 0; i < HD; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int i = 0; i < 64; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if (done_ok && row_valid) {
-      const float lse = (l_run > 0.0f) ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+    if (done_ok && row_valid && hf == 0) {
+      const float lse = (l_tot > 0.0f) ? (m_run + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
       p.lse_part[out_row * p.n_h + head] = lse;
     }
   }
