@@ -30,8 +30,8 @@
 //              overlaps the other tile's MMAs (ping-pong).
 // Two threads per row halve the latency of a softmax step, which otherwise
 // exceeds the MMA time of one tile and stalls the ping-pong.
-// TMEM (512 columns): S_a 0, S_b 128 (P over the first 64 columns), O_a 256,
-// O_b 384. tcgen05 operations of one thread complete in issue order, so the
+// TMEM (512 columns): S_a 0, S_b 128, O_a 256, O_b 384. Each half row's P
+// (bf16 pairs) goes over the first 32 of its own 64 S columns. tcgen05 operations of one thread complete in issue order, so the
 // completion of S_x(j+1) also means O_x += P_x(j) V_j has completed.
 #pragma once
 
@@ -116,6 +116,61 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint3
       return;
     }
   }
+}
+
+// Exponentials of one half row (64 keys) for one KV tile: P = 2^(S*scale*log2e - m)
+// as bf16 pairs over the first 32 of the half row's S columns, returning the
+// sum of the fp32 values. The S half is read again from TMEM 16 columns at a
+// time, the next chunk in flight while this one is exponentiated (P chunk h8,
+// columns 8h8.., lies below every S chunk not yet read). kPolyPairsPer8 of
+// every 8 pairs take the polynomial on the FMA pipe, the rest the special
+// function unit. kMasked: keys past `lim` are hidden and get exactly 0 (the
+// polynomial or a large unmasked S would leave a value there); a separate
+// instantiation keeps the compares out of the unmasked tiles.
+template <bool kMasked>
+__device__ __forceinline__ float half_row_exps(uint32_t s_col, float sl2, float m_use, int lim) {
+  const uint64_t sl2_2 = f2_pack(sl2, sl2);
+  const uint64_t negm_2 = f2_pack(-m_use, -m_use);
+  uint64_t acc[2] = {0ull, 0ull};
+  uint32_t sc[2][16];
+  tmem_ld16(s_col, sc[0]);
+  tmem_ld_wait();
+#pragma unroll
+  for (int h8 = 0; h8 < 4; ++h8) {
+    if (h8 < 3) tmem_ld16(s_col + (h8 + 1) * 16, sc[(h8 + 1) & 1]);
+    const uint32_t (&sv)[16] = sc[h8 & 1];
+    uint32_t pk[8];
+#pragma unroll
+    for (int cc = 0; cc < 16; cc += 2) {
+      const int c = h8 * 16 + cc;
+      const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[cc]), __uint_as_float(sv[cc + 1])), sl2_2, negm_2);
+      uint64_t p2;
+      if (((c >> 1) & 7) < kPolyPairsPer8) {
+        p2 = exp2_poly_x2(x2);
+      } else {
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        p2 = f2_pack(ex2(x0), ex2(x1));
+      }
+      if (kMasked) {
+        float p0, p1;
+        f2_unpack(p2, p0, p1);
+        if (c > lim) p0 = 0.0f;
+        if (c + 1 > lim) p1 = 0.0f;
+        p2 = f2_pack(p0, p1);
+      }
+      float p0, p1;
+      f2_unpack(p2, p0, p1);
+      pk[cc >> 1] = pack_bf16x2(p0, p1);
+      acc[(c >> 1) & 1] = f2_add(acc[(c >> 1) & 1], p2);
+    }
+    tmem_st8(s_col + h8 * 8, pk);
+    if (h8 < 3) tmem_ld_wait();
+  }
+  const uint64_t t = f2_add(acc[0], acc[1]);
+  float lo, hi;
+  f2_unpack(t, lo, hi);
+  return lo + hi;
 }
 
 // 18 warps put five on two of the four schedulers, whose register files hold
@@ -242,7 +297,9 @@ __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Para
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           const uint64_t b = umma_sdesc_sw128(v_addr + (j % kVStages) * kTileBytes + kk * 2048, kHalfBytes, 1024);
-          umma_bf16_ts(tmem + kColO + x * HD, tmem + kColS + x * BN + kk * 8, b, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          // keys 16kk..16kk+15 as bf16 pairs: the P of each half sits in its own first 32 S columns
+          const uint32_t p_addr = tmem + kColS + x * BN + (kk >> 2) * 64 + (kk & 3) * 8;
+          umma_bf16_ts(tmem + kColO + x * HD, p_addr, b, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&bars[B_O_DONE + x]);
       };
@@ -281,7 +338,6 @@ __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Para
     const int row = quarter * 32 + lane;    // packed row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_col = tmem + lane_base + kColS + x * BN + hf * 64;   // this thread's S columns
-    const uint32_t p_col = tmem + lane_base + kColS + x * BN + hf * 32;   // its P columns (bf16 pairs)
     const uint32_t o_col = tmem + lane_base + kColO + x * HD + hf * 64;   // its O columns
     float* xch_mine = reinterpret_cast<float*>(smem + kOffXch) + (x * 2 + hf) * BM + row;
     const float* xch_peer = reinterpret_cast<const float*>(smem + kOffXch) + (x * 2 + (hf ^ 1)) * BM + row;
@@ -338,9 +394,6 @@ __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Para
         // KV tile and agree on whether to go on, so neither can wait alone.
         // The peer reads this slot before it arrives on P_FULL, and the next
         // write comes after S_FULL, which needs that arrival: no overwrite race.
-        // The barrier also orders the partner's completed S loads before this
-        // thread's P stores, which overwrite S columns 32-63 (the tcgen05
-        // fences carry that order across the thread sync).
         *xch_mine = mx;
         tc_fence_before();
         if (!named_bar_and(pair_bar, 64, got)) { ok = false; break; }
@@ -356,51 +409,9 @@ __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Para
           resc = true;
         }
         const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
-        // p = 2^(s * scale * log2 e - m) in packed pairs: kPolyPairsPer8 of every
-        // 8 pairs through the polynomial on the FMA pipe, the rest through the
-        // special-function unit. P goes back over the S row as bf16 pairs, 8
-        // columns (16 keys) at a time; the row sum runs in two packed chains.
-        const uint64_t sl2_2 = f2_pack(sl2, sl2);
-        const uint64_t negm_2 = f2_pack(-m_use, -m_use);
-        uint64_t acc[2] = {0ull, 0ull};
-#pragma unroll
-        for (int h8 = 0; h8 < 4; ++h8) {
-          uint32_t pk[8];
-#pragma unroll
-          for (int cc = 0; cc < 16; cc += 2) {
-            const int c = h8 * 16 + cc;
-            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[c >> 5][c & 31]), __uint_as_float(s[c >> 5][(c + 1) & 31])),
-                                       sl2_2, negm_2);
-            uint64_t p2;
-            if (((c >> 1) & 7) < kPolyPairsPer8) {
-              p2 = exp2_poly_x2(x2);
-              // hidden keys contribute exactly zero (the polynomial leaves a tiny value there)
-              if (lim < 63) {
-                float p0, p1;
-                f2_unpack(p2, p0, p1);
-                if (c > lim) p0 = 0.0f;
-                if (c + 1 > lim) p1 = 0.0f;
-                p2 = f2_pack(p0, p1);
-              }
-            } else {
-              float x0, x1;
-              f2_unpack(x2, x0, x1);
-              p2 = f2_pack(ex2(x0), ex2(x1));   // ex2(-inf) is exactly 0
-            }
-            float p0, p1;
-            f2_unpack(p2, p0, p1);
-            pk[cc >> 1] = pack_bf16x2(p0, p1);
-            acc[(c >> 1) & 1] = f2_add(acc[(c >> 1) & 1], p2);
-          }
-          tmem_st8(p_col + h8 * 8, pk);
-        }
-        float sum;
-        {
-          const uint64_t t = f2_add(acc[0], acc[1]);
-          float lo, hi;
-          f2_unpack(t, lo, hi);
-          sum = lo + hi;
-        }
+        const bool tile_masked = __any_sync(0xffffffffu, lim < 63);
+        const float sum = tile_masked ? half_row_exps<true>(s_col, sl2, m_use, lim)
+                                      : half_row_exps<false>(s_col, sl2, m_use, lim);
         l_run = l_run * alpha + sum;
         // O_x holds every earlier PV (see S_FULL above): rescale this half in place if needed
         if (it > 0 && __any_sync(0xffffffffu, resc)) {
