@@ -70,7 +70,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;     // + tile * 128
 constexpr uint32_t kColO = 256;   // + tile * 128
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled when the max grows by > 2^8
-constexpr int kPolyPairsPer8 = 2;          // of every 8 column pairs, this many take the polynomial exp2
+constexpr int kPolyPairsPer8 = 1;          // of every 8 column pairs, this many take the polynomial exp2
 
 // barrier slots
 enum {
@@ -280,26 +280,30 @@ __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Para
     if (lane == 0 && n_iter > 0) {
       constexpr uint32_t idesc_s = umma_idesc_bf16(BM, BN, 0);   // Q, K both K-major
       constexpr uint32_t idesc_o = umma_idesc_bf16(BM, HD, 1);   // P (TMEM) K-major, V MN-major
-      const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t k_addr = smem_u32(sK);
-      const uint32_t v_addr = smem_u32(sV);
+      // Descriptors of the tile bases; an operand at byte offset `off` from a
+      // base is base + off/16 (the 14-bit address field does not carry: every
+      // shared address is below 256 KB).
+      const uint64_t q_desc = umma_sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t k_desc = umma_sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t v_desc = umma_sdesc_sw128(smem_u32(sV), kHalfBytes, 1024);
       auto issue_s = [&](int x, int i) {   // S_x(i) = Q_x K_i^T
+        const uint64_t qd = q_desc + static_cast<uint64_t>((x * kTileBytes) >> 4);
+        const uint64_t kd = k_desc + static_cast<uint64_t>(((i % kKStages) * kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          const uint64_t a = umma_sdesc_sw128(q_addr + x * kTileBytes + off, 16, 1024);
-          const uint64_t b = umma_sdesc_sw128(k_addr + (i % kKStages) * kTileBytes + off, 16, 1024);
-          umma_bf16_ss(tmem + kColS + x * BN, a, b, idesc_s, kk > 0 ? 1u : 0u);
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
+          umma_bf16_ss(tmem + kColS + x * BN, qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(&bars[B_S_FULL + x]);
       };
       auto issue_pv = [&](int x, int j) {  // O_x += P_x(j) V_j
+        const uint64_t vd = v_desc + static_cast<uint64_t>(((j % kVStages) * kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t b = umma_sdesc_sw128(v_addr + (j % kVStages) * kTileBytes + kk * 2048, kHalfBytes, 1024);
           // keys 16kk..16kk+15 as bf16 pairs: the P of each half sits in its own first 32 S columns
           const uint32_t p_addr = tmem + kColS + x * BN + (kk >> 2) * 64 + (kk & 3) * 8;
-          umma_bf16_ts(tmem + kColO + x * HD, p_addr, b, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts(tmem + kColO + x * HD, p_addr, vd + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o,
+                       (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&bars[B_O_DONE + x]);
       };
