@@ -43,7 +43,7 @@ EXPORTED = (
     "cp_status_string", "cp_abi_version", "cp_shard_plan", "cp_rank_ranges", "cp_ring_schedule",
     "cp_classify_pair", "cp_block_pairs", "cp_ring_comm_volume", "cp_workspace_size",
     "cp_reset_status", "cp_check_status", "cp_attn_partial", "cp_attn_merge", "cp_decode",
-    "cp_decode_static",
+    "cp_decode_static", "cp_decode_partial",
 )
 
 
@@ -99,6 +99,7 @@ def lib() -> ctypes.CDLL:
         "cp_attn_merge": (i32, [vp, vp, i32, i64, i64, i32, i32, vp, i32, vp, vp]),
         "cp_decode": (i32, [vp, vp, vp, i32, vp, i32, i64, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]),
         "cp_decode_static": (i32, [vp, vp, vp, i32, vp, i32, i64, i32, i32, i32, i32, f32, vp, vp, vp]),
+        "cp_decode_partial": (i32, [vp, vp, vp, i32, vp, i32, i64, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -241,6 +242,17 @@ def cp_decode(q, k, v, kv_offsets, n_h: int, n_kv: int, n_splits: int, softmax_s
                            _ptr(out), _ptr(lse_out), _ptr(workspace),
                            int(workspace.numel() * workspace.element_size()), _stream(stream))
     _check("cp_decode", code)
+
+
+def cp_decode_partial(q, k, v, kv_offsets, n_h: int, n_kv: int, n_splits: int, softmax_scale: float, o_part,
+                      lse_part, workspace, stream=None) -> None:
+    """cp_decode's partial: o_part [batch, n_h, d] fp32 and lse_part [batch, n_h]
+    fp32 over the keys k/v hold, for a later cp_attn_merge across ranks."""
+    code = lib().cp_decode_partial(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(kv_offsets), int(q.shape[0]),
+                                   int(k.shape[0]), n_h, n_kv, int(q.shape[-1]), n_splits, float(softmax_scale),
+                                   _ptr(o_part), _ptr(lse_part), _ptr(workspace),
+                                   int(workspace.numel() * workspace.element_size()), _stream(stream))
+    _check("cp_decode_partial", code)
 
 
 def cp_decode_static(q, k, v, kv_offsets, n_h: int, n_kv: int, n_splits: int, softmax_scale: float, out, lse_out,

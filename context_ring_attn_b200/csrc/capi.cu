@@ -390,9 +390,9 @@ cp_status cp_attn_merge(const float* o_parts, const float* lse_parts, int32_t n_
   return last_cuda_status();
 }
 
-cp_status cp_decode(const void* q, const void* k, const void* v, cp_dtype dtype, const int64_t* kv_offsets,
+static cp_status decode_impl(const void* q, const void* k, const void* v, cp_dtype dtype, const int64_t* kv_offsets,
                     int32_t batch, int64_t kv_rows, int32_t n_h, int32_t n_kv, int32_t d, int32_t n_splits,
-                    float softmax_scale, void* out, float* lse_out, void* workspace, size_t ws_bytes,
+                    float softmax_scale, void* out, bool out_f32, float* lse_out, void* workspace, size_t ws_bytes,
                     void* cuda_stream) {
   if (!q || !k || !v || !kv_offsets || !out) return CP_ERR_INVALID_ARG;
   if (batch < 0 || kv_rows < 0 || n_h < 1 || n_kv < 1 || d < 1 || n_h % n_kv) return CP_ERR_INVALID_ARG;
@@ -400,7 +400,7 @@ cp_status cp_decode(const void* q, const void* k, const void* v, cp_dtype dtype,
   if (n_splits < 1 || n_splits > dec::kMaxSplits) return CP_ERR_UNSUPPORTED;
   const int group = n_h / n_kv;
   if (dtype != CP_BF16 || d != 128 || group > 16 || (16 % group) != 0) return CP_ERR_UNSUPPORTED;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 8) || !aligned(kv_offsets, 8))
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, out_f32 ? 16 : 8) || !aligned(kv_offsets, 8))
     return CP_ERR_INVALID_ARG;
   if (!workspace || !aligned(workspace, 256) || ws_bytes < decode_ws_bytes(dec::kWarps, batch, n_h, n_kv, d))
     return CP_ERR_WORKSPACE;   // below what even the smallest grid needs
@@ -434,9 +434,30 @@ cp_status cp_decode(const void* q, const void* k, const void* v, cp_dtype dtype,
   dec::decode_split_kernel<<<static_cast<unsigned>(n_warps / dec::kWarps), dec::kThreads, dec::kSmemBytes, stream>>>(p);
   if (last_cuda_status() != CP_OK) return CP_ERR_CUDA;
   const int64_t n_rowheads = static_cast<int64_t>(batch) * n_h;
-  dec::decode_merge_kernel<<<static_cast<unsigned>(n_rowheads), dec::kMergeThreads, 0, stream>>>(
-      p, static_cast<__nv_bfloat16*>(out), lse_out);
+  if (out_f32)
+    dec::decode_merge_kernel<float><<<static_cast<unsigned>(n_rowheads), dec::kMergeThreads, 0, stream>>>(
+        p, static_cast<float*>(out), lse_out);
+  else
+    dec::decode_merge_kernel<__nv_bfloat16><<<static_cast<unsigned>(n_rowheads), dec::kMergeThreads, 0, stream>>>(
+        p, static_cast<__nv_bfloat16*>(out), lse_out);
   return last_cuda_status();
+}
+
+cp_status cp_decode(const void* q, const void* k, const void* v, cp_dtype dtype, const int64_t* kv_offsets,
+                    int32_t batch, int64_t kv_rows, int32_t n_h, int32_t n_kv, int32_t d, int32_t n_splits,
+                    float softmax_scale, void* out, float* lse_out, void* workspace, size_t ws_bytes,
+                    void* cuda_stream) {
+  return decode_impl(q, k, v, dtype, kv_offsets, batch, kv_rows, n_h, n_kv, d, n_splits, softmax_scale, out, false,
+                     lse_out, workspace, ws_bytes, cuda_stream);
+}
+
+cp_status cp_decode_partial(const void* q, const void* k, const void* v, cp_dtype dtype, const int64_t* kv_offsets,
+                            int32_t batch, int64_t kv_rows, int32_t n_h, int32_t n_kv, int32_t d, int32_t n_splits,
+                            float softmax_scale, float* o_part, float* lse_part, void* workspace, size_t ws_bytes,
+                            void* cuda_stream) {
+  if (!lse_part) return CP_ERR_INVALID_ARG;
+  return decode_impl(q, k, v, dtype, kv_offsets, batch, kv_rows, n_h, n_kv, d, n_splits, softmax_scale, o_part, true,
+                     lse_part, workspace, ws_bytes, cuda_stream);
 }
 
 }  // extern "C"

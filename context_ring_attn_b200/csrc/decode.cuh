@@ -364,8 +364,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
 constexpr int kMergeThreads = 256;
 constexpr int kMergeUnroll = 4;
 
+__device__ __forceinline__ void store_row4(__nv_bfloat16* dst, float4 v) {
+  uint2 u;
+  u.x = pack_bf16x2(v.x, v.y);
+  u.y = pack_bf16x2(v.z, v.w);
+  *reinterpret_cast<uint2*>(dst) = u;
+}
+__device__ __forceinline__ void store_row4(float* dst, float4 v) { *reinterpret_cast<float4*>(dst) = v; }
+
+// OutT: bf16 for the decoded output, float for a partial (O, LSE) that a
+// later LSE merge combines with other ranks' partials.
+template <typename OutT>
 __global__ void __launch_bounds__(kMergeThreads, 4) decode_merge_kernel(const __grid_constant__ Params p,
-                                                                      __nv_bfloat16* out, float* lse_out) {
+                                                                      OutT* out, float* lse_out) {
   __shared__ float sm_m[8], sm_l[8];
   __shared__ float4 sm_o[8][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -450,10 +461,7 @@ __global__ void __launch_bounds__(kMergeThreads, 4) decode_merge_kernel(const __
       }
     }
     const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
-    uint2 u;
-    u.x = pack_bf16x2(o.x * inv, o.y * inv);
-    u.y = pack_bf16x2(o.z * inv, o.w * inv);
-    *reinterpret_cast<uint2*>(out + rh * 128 + lane * 4) = u;
+    store_row4(out + rh * 128 + lane * 4, make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv));
     if (lse_out && lane == 0) lse_out[rh] = (L > 0.0f) ? M + logf(L) : -INFINITY;
   }
 }

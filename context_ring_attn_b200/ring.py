@@ -105,3 +105,66 @@ def run_ring(sched: RingSchedule, q, k, v, n_h: int, n_kv: int, out, lse_out=Non
     else:
         raise ValueError(merge)
     return out
+
+
+class DecodeCP:
+    """Context-parallel decode over N virtual ranks.
+
+    "Context Parallelism for Scalable Million-Token Inference", section 3:
+    in decode each CP rank holds a shard of every request's KV cache (the
+    shards the prefill's plan gave it) and the queries travel the ring
+    (pass-Q); after N steps every rank has decoded every query against its own
+    shard, an all-to-all returns the partials (O, LSE) to the queries' owners
+    and they are merged. On one GPU the N^2 (rank, query shard) visits of the
+    ring are one batched cp_decode_partial launch over "virtual requests"
+    (rank r, request b) in rank-major order, so the partial of rank r for
+    request b lands at row r*B + b: the all-to-all is that index, and
+    cp_attn_merge over the N parts finishes the decode. The shards are
+    gathered once at construction (each rank's own cache in a real
+    deployment); the arithmetic runs in the library's kernels.
+    """
+
+    def __init__(self, k, v, offsets_host, n_ranks: int, mode: int = B.CP_SHARD_LOAD_BALANCED):
+        offsets_host = [int(x) for x in offsets_host]
+        n_req = len(offsets_host) - 1
+        self.n_ranks, self.n_req = n_ranks, n_req
+        segs = B.segments([(offsets_host[b + 1] - offsets_host[b], offsets_host[b], 0, b) for b in range(n_req)])
+        idx, offs = [], [0]
+        for r in range(n_ranks):
+            per_req = [[] for _ in range(n_req)]
+            for g in B.cp_rank_ranges(segs, n_req, n_ranks, mode, r):
+                per_req[g.seq].append(g)
+            for b in range(n_req):
+                n = 0
+                for g in per_req[b]:
+                    if g.len > 0:
+                        idx.append(torch.arange(g.row0, g.row0 + g.len, dtype=torch.int64))
+                        n += g.len
+                offs.append(offs[-1] + n)
+        rows = torch.cat(idx) if idx else torch.zeros(0, dtype=torch.int64)
+        if rows.numel() == 0:   # no keys anywhere: one unused row keeps the buffers non-empty
+            rows = torch.zeros(1, dtype=torch.int64)
+        rows = rows.to(k.device)
+        self.k = k.index_select(0, rows)
+        self.v = v.index_select(0, rows)
+        self.offsets = torch.tensor(offs, dtype=torch.int64, device=k.device)
+        self.kv_bytes = 2 * (offs[-1] * int(k.shape[1]) * int(k.shape[2]) * k.element_size())
+
+    def buffers(self, q, n_splits: int):
+        """Partial buffers, the per-rank query copies and a decode workspace."""
+        n, n_req = self.n_ranks, self.n_req
+        n_h, d = int(q.shape[1]), int(q.shape[2])
+        o_parts = torch.empty((n * n_req, n_h, d), dtype=torch.float32, device=q.device)
+        lse_parts = torch.empty((n * n_req, n_h), dtype=torch.float32, device=q.device)
+        ws = torch.zeros(B.cp_workspace_size(B.CP_OP_DECODE, n * n_req, n_h, d, n_splits), dtype=torch.uint8,
+                         device=q.device)
+        return o_parts, lse_parts, ws
+
+    def run(self, q_ranks, n_kv: int, n_splits: int, softmax_scale: float, out, lse_out, o_parts, lse_parts,
+            workspace, stream=None):
+        """q_ranks: the queries as every rank holds them, [N*B, n_h, d] (q repeated
+        N times, rank-major). out [B, n_h, d] bf16, lse_out [B, n_h] fp32."""
+        n_h, d = int(q_ranks.shape[1]), int(q_ranks.shape[2])
+        B.cp_decode_partial(q_ranks, self.k, self.v, self.offsets, n_h, n_kv, n_splits, softmax_scale,
+                            o_parts, lse_parts, workspace, stream)
+        B.cp_attn_merge(o_parts, lse_parts, self.n_ranks, self.n_req, self.n_req, n_h, d, out, lse_out, stream)

@@ -242,6 +242,21 @@ cp_status cp_decode(const void* q, const void* k, const void* v, cp_dtype dtype,
                     int32_t n_kv, int32_t d, int32_t n_splits, float softmax_scale, void* out,
                     float* lse_out, void* workspace, size_t ws_bytes, void* cuda_stream);
 
+/* The decode of cp_decode as a partial: O (fp32, normalised over the keys this
+ * call sees) and its LSE, for context-parallel decode, where every rank holds
+ * a shard of each request's KV cache, decodes the queries against its shard
+ * and the per-rank partials are merged with cp_attn_merge (method page,
+ * section 3: ring pass-Q for decode; the merge after the final all-to-all is
+ * the "merge attention" step of section 5). Arguments, limits and workspace as
+ * in cp_decode, with o_part [batch, n_h, d] fp32 (16-byte aligned) in place of
+ * out and lse_part [batch, n_h] fp32 required. A request with no keys here
+ * yields O = 0, LSE = -inf, which the merge weighs 0. */
+cp_status cp_decode_partial(const void* q, const void* k, const void* v, cp_dtype dtype,
+                            const int64_t* kv_offsets, int32_t batch, int64_t kv_rows, int32_t n_h,
+                            int32_t n_kv, int32_t d, int32_t n_splits, float softmax_scale,
+                            float* o_part, float* lse_part, void* workspace, size_t ws_bytes,
+                            void* cuda_stream);
+
 /* Split-KV decode for callers that cannot allocate device memory when they
  * decode (code inside an allocator or memory pool, plugins that are given only
  * their inputs and outputs, serving loops that forbid allocation after

@@ -212,3 +212,66 @@ def test_decode_reports_decreasing_offsets():
     with pytest.raises(B.CpError) as e:
         B.cp_check_status(ws)
     assert e.value.code == B.CP_ERR_INTERNAL
+
+
+# ---------------------------------------------------------------------------- decode partials, CP decode, graphs
+def _decode_case(lens, n_h, n_kv, seed):
+    dc = synth.make_decode(len(lens), n_h, n_kv, 128, lens, seed, 0.5)
+    return dc, dev(dc.q_raw, "bf16"), dev(dc.k_raw, "bf16"), dev(dc.v_raw, "bf16"), torch.from_numpy(dc.offsets).cuda()
+
+
+def test_decode_partial_matches_oracle():
+    lens = [0, 7, 129, 2000, 64]
+    dc, q, k, v, off = _decode_case(lens, 16, 2, 61)
+    o = torch.empty((len(lens), 16, 128), dtype=torch.float32, device="cuda")
+    lse = torch.empty((len(lens), 16), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(B.cp_workspace_size(B.CP_OP_DECODE, len(lens), 16, 128, 32), dtype=torch.uint8, device="cuda")
+    B.cp_decode_partial(q, k, v, off, 16, 2, 32, 1 / math.sqrt(128), o, lse, ws)
+    B.cp_check_status(ws)
+    o_ref, l_ref = OD.decode(dc.q, dc.k, dc.v, dc.offsets)
+    check(o.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "bf16", "decode partial")
+
+
+@pytest.mark.parametrize("n_ranks,mode", [(2, B.CP_SHARD_LOAD_BALANCED), (4, B.CP_SHARD_LOAD_BALANCED),
+                                          (8, B.CP_SHARD_CONTIGUOUS), (8, B.CP_SHARD_LOAD_BALANCED)])
+def test_decode_context_parallel(n_ranks, mode):
+    """Every rank decodes every query against its shard of the cache; the merged
+    partials equal the decode of the whole cache."""
+    lens = [0, 5, 100, 255, 256, 1000, 3001, 64, 17]
+    dc, q, k, v, off = _decode_case(lens, 16, 1, 70 + n_ranks)
+    cp = ring.DecodeCP(k, v, dc.offsets, n_ranks, mode)
+    o_parts, lse_parts, ws = cp.buffers(q, 16)
+    q_ranks = q.repeat(n_ranks, 1, 1)
+    out = torch.empty((len(lens), 16, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((len(lens), 16), dtype=torch.float32, device="cuda")
+    cp.run(q_ranks, 1, 16, 1 / math.sqrt(128), out, lse, o_parts, lse_parts, ws)
+    B.cp_check_status(ws)
+    o_ref, l_ref = OD.decode(dc.q, dc.k, dc.v, dc.offsets)
+    check(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "bf16", "cp decode")
+
+
+def test_decode_replays_from_a_cuda_graph():
+    """cp_decode captured once (after one eager call) and replayed on new
+    inputs copied into the captured buffers gives the eager results."""
+    lens = [300, 4096, 77, 1500]
+    dc, q, k, v, off = _decode_case(lens, 16, 1, 81)
+    dc2, q2, k2, v2, _ = _decode_case(lens, 16, 1, 82)
+    out = torch.empty((4, 16, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((4, 16), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(B.cp_workspace_size(B.CP_OP_DECODE, 4, 16, 128, 64), dtype=torch.uint8, device="cuda")
+    scale = 1 / math.sqrt(128)
+    B.cp_decode(q, k, v, off, 16, 1, 64, scale, out, lse, ws)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        B.cp_decode(q, k, v, off, 16, 1, 64, scale, out, lse, ws)
+    g.replay()
+    torch.cuda.synchronize()
+    o_ref, l_ref = OD.decode(dc.q, dc.k, dc.v, dc.offsets)
+    check(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "bf16", "graph replay")
+    q.copy_(q2), k.copy_(k2), v.copy_(v2)
+    g.replay()
+    torch.cuda.synchronize()
+    B.cp_check_status(ws)
+    o_ref2, l_ref2 = OD.decode(dc2.q, dc2.k, dc2.v, dc2.offsets)
+    check(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref2, l_ref2, "bf16", "graph replay, new inputs")

@@ -128,3 +128,28 @@ def test_random_pairs_against_reference():
         for causal in (True, False):
             assert B.cp_classify_pair(q, k, causal) == OP.pair_class(oq, ok, causal)
             assert B.cp_block_pairs(ranges, blk, causal) == OP.visible_pairs(oq, ok, causal)
+
+
+@pytest.mark.parametrize("n_ranks,mode", [(2, B.CP_SHARD_LOAD_BALANCED), (8, B.CP_SHARD_LOAD_BALANCED),
+                                          (3, B.CP_SHARD_CONTIGUOUS)])
+def test_decode_shards_partition_every_request(n_ranks, mode):
+    """The per-rank decode shards hold every key of every request exactly once,
+    in request order within each rank, with CSR offsets per (rank, request)."""
+    import torch
+    from context_ring_attn_b200 import ring
+    lens = [0, 5, 100, 31, 256, 1000]
+    offsets = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    total = int(offsets[-1])
+    k = torch.arange(total, dtype=torch.float32).reshape(total, 1, 1)   # row id as the value
+    cp = ring.DecodeCP(k, k, offsets, n_ranks, mode)
+    offs = cp.offsets.numpy()
+    assert offs.shape == (n_ranks * len(lens) + 1,) and offs[0] == 0
+    assert np.all(np.diff(offs) >= 0)
+    seen = np.zeros(total, dtype=np.int64)
+    for r in range(n_ranks):
+        for b in range(len(lens)):
+            i = r * len(lens) + b
+            rows = cp.k[offs[i]:offs[i + 1], 0, 0].numpy().astype(np.int64)
+            assert np.all((rows >= offsets[b]) & (rows < offsets[b + 1]))
+            seen[rows] += 1
+    assert np.all(seen == 1)
