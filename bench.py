@@ -570,6 +570,91 @@ def run_decode(args, dev):
                             "then the 8-way LSE merge"}}
 
 
+SWEEP_MISS = (0.01, 0.025, 0.0325, 0.05, 0.10, 0.20, 0.50, 1.00)
+SWEEP_LINKS = {"rdma_400gbps": 50e9, "nvlink_peer_measured": 770e9}
+
+
+def run_sweep(args, dev):
+    """Algorithm 1 sweep: persistent-KV prefill with T + P = 128000 (128/8
+    heads, D_H 128, bf16, 8 virtual ranks) at the method page's miss rates.
+    Per point and variant, the GPU time of the whole ring schedule (all N^2
+    blocks, running 2-way merges) is measured on one GPU; a rank of an N-GPU
+    ring does 1/N of it and 1/N^2 per ring step. The ring's exposed transfer
+    is modelled per link: pass-KV (N-1) hops of a KV shard, each hidden under
+    a step up to its length; pass-Q (N-1) hops of a Q shard likewise, plus the
+    all-to-all of the fp32 partials (not overlapped). The selector is
+    cp_select_ring_variant fed the measured step time."""
+    import torch
+
+    from context_ring_attn_b200 import binding as B
+    from context_ring_attn_b200 import ring, synth
+
+    n_h, n_kv, d, n, total = 128, 8, 128, 8, 128000
+    scale = 1.0 / math.sqrt(d)
+    seed = synth.WORKLOADS["persistent_kv"]["seed"]
+    q_all = synth.device_rows(seed, synth.TENSOR_Q, total, (n_h, d), 0.5, "bf16", dev)
+    k = synth.device_rows(seed, synth.TENSOR_K, total, (n_kv, d), 0.5, "bf16", dev)
+    v = synth.device_rows(seed, synth.TENSOR_V, total, (n_kv, d), 0.5, "bf16", dev)
+    o_all = torch.empty((2 * total, n_h, d), dtype=torch.float32, device=dev)
+    l_all = torch.empty((2 * total, n_h), dtype=torch.float32, device=dev)
+    out_all = torch.empty((total, n_h, d), dtype=torch.bfloat16, device=dev)
+    lse_all = torch.empty((total, n_h), dtype=torch.float32, device=dev)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    points = []
+    for miss in SWEEP_MISS:
+        t = int(round(miss * total))
+        p = total - t
+        q = q_all[:t]
+        q_segs = [ring.Segment(t, 0, p, 0)]
+        kv_segs = [ring.Segment(p, 0, 0, 0), ring.Segment(t, p, p, 0)] if p > 0 else [ring.Segment(t, 0, 0, 0)]
+        res = {"miss_rate": miss, "T": t, "P": p}
+        for name, variant in (("pass_kv", B.CP_PASS_KV), ("pass_q", B.CP_PASS_Q)):
+            sched = ring.RingSchedule(q_segs, kv_segs, n, variant)
+
+            def once():
+                ring.run_ring(sched, q, k, v, n_h, n_kv, out_all[:t], lse_all[:t], True, scale,
+                              o_all[:2 * t], l_all[:2 * t], ws, merge="running")
+            once()
+            reps = 3
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                once()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            res[name + "_gpu_ms"] = e0.elapsed_time(e1) / reps
+        B.cp_check_status(ws)
+        flops = 4.0 * d * n_h * (t * p + t * (t + 1) / 2)
+        res["tflop"] = flops / 1e12
+        res["links"] = {}
+        for lname, bw in SWEEP_LINKS.items():
+            r = {}
+            for name in ("pass_kv", "pass_q"):
+                rank_ms = res[name + "_gpu_ms"] / n
+                step_ms = rank_ms / n
+                if name == "pass_kv":
+                    hop_ms = (t + p) / n * n_kv * d * 2 * 2 / bw * 1e3
+                    a2a_ms = 0.0
+                else:
+                    hop_ms = t / n * n_h * d * 2 / bw * 1e3
+                    a2a_ms = (n - 1) * (t / n) * n_h * (d + 1) * 4 / bw * 1e3
+                r[name + "_ms"] = rank_ms + (n - 1) * max(0.0, hop_ms - step_ms) + a2a_ms
+            step_kv_s = res["pass_kv_gpu_ms"] / n / n * 1e-3
+            var, why = B.cp_select_ring_variant(t, p, n_h, n_kv, d, n, 2, bw, step_kv_s)
+            r["faster"] = "pass_kv" if r["pass_kv_ms"] <= r["pass_q_ms"] else "pass_q"
+            r["selected"] = "pass_kv" if var == B.CP_PASS_KV else "pass_q"
+            r["selector_condition"] = why
+            res["links"][lname] = r
+        points.append(res)
+    del q_all, k, v, o_all, l_all, out_all, lse_all
+    torch.cuda.empty_cache()
+    return {"workload": "persistent-KV prefill, T+P=128000, N_H=128, N_KV=8, D_H=128, bf16, 8 virtual ranks",
+            "links_bytes_per_s": SWEEP_LINKS, "points": points,
+            "note": "gpu_ms: whole ring schedule on one GPU (measured); per-link totals are one rank of an "
+                    "8-GPU ring (measured compute / 8 + modelled exposed transfer)"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -582,6 +667,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-secondary", action="store_true", help="skip the persistent-KV and varlen workloads")
     ap.add_argument("--only-decode", action="store_true", help="time the split-KV decode workload alone")
+    ap.add_argument("--sweep-miss-rate", action="store_true",
+                    help="Algorithm 1 sweep of pass-KV vs pass-Q over KV-cache miss rates (prints its own line)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="shorter sequence for profiling captures (default: the full 131072)")
     args = ap.parse_args()
@@ -604,6 +691,10 @@ def main():
     try:
         if args.only_decode:
             print(json.dumps({"decode": run_decode(args, torch.device("cuda", local))}), flush=True)
+            return
+        if args.sweep_miss_rate:
+            if rank == 0:
+                print(json.dumps({"sweep": run_sweep(args, torch.device("cuda", local))}), flush=True)
             return
         run_ours(args, rank, world)
     finally:

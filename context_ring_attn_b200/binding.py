@@ -43,7 +43,7 @@ EXPORTED = (
     "cp_status_string", "cp_abi_version", "cp_shard_plan", "cp_rank_ranges", "cp_ring_schedule",
     "cp_classify_pair", "cp_block_pairs", "cp_ring_comm_volume", "cp_workspace_size",
     "cp_reset_status", "cp_check_status", "cp_attn_partial", "cp_attn_merge", "cp_decode",
-    "cp_decode_static", "cp_decode_partial",
+    "cp_decode_static", "cp_decode_partial", "cp_select_ring_variant",
 )
 
 
@@ -99,6 +99,8 @@ def lib() -> ctypes.CDLL:
         "cp_attn_merge": (i32, [vp, vp, i32, i64, i64, i32, i32, vp, i32, vp, vp]),
         "cp_decode": (i32, [vp, vp, vp, i32, vp, i32, i64, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]),
         "cp_decode_static": (i32, [vp, vp, vp, i32, vp, i32, i64, i32, i32, i32, i32, f32, vp, vp, vp]),
+        "cp_select_ring_variant": (i32, [i64, i64, i32, i32, i32, i32, i32, ctypes.c_double, ctypes.c_double,
+                                          vp, vp]),
         "cp_decode_partial": (i32, [vp, vp, vp, i32, vp, i32, i64, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
@@ -182,6 +184,18 @@ def cp_ring_schedule(q_segs, n_q_seg: int, kv_segs, n_kv_seg: int, n_ranks: int,
     _check("cp_ring_schedule", lib().cp_ring_schedule(q_segs, n_q_seg, kv_segs, n_kv_seg, n_ranks, mode, variant,
                                                       ranges, cap, ctypes.byref(n), blocks, parts))
     return ranges, n.value, blocks, list(parts)
+
+
+def cp_select_ring_variant(t: int, p: int, n_h: int, n_kv: int, d: int, n_ranks: int, elem_bytes: int,
+                           link_bytes_per_s: float, step_attn_s: float):
+    """Algorithm 1: returns (variant, reason) with reason 1 or 2 for the
+    condition that chose pass-KV and 0 for pass-Q."""
+    var = ctypes.c_int32(-1)
+    why = ctypes.c_int32(-1)
+    _check("cp_select_ring_variant", lib().cp_select_ring_variant(
+        t, p, n_h, n_kv, d, n_ranks, elem_bytes, float(link_bytes_per_s), float(step_attn_s), ctypes.byref(var),
+        ctypes.byref(why)))
+    return var.value, why.value
 
 
 def cp_classify_pair(q: cp_range, kv: cp_range, causal: bool = True) -> int:

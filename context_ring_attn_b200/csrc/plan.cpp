@@ -222,4 +222,28 @@ cp_status cp_ring_comm_volume(const cp_range* ranges, const cp_block* blocks, in
   return CP_OK;
 }
 
+// Algorithm 1 of the method page (section 3): pass-KV when the KV-cache miss
+// rate T/(T+P) is above 2*N_KV/N_H, or when one ring hop's SendRecv of a KV
+// shard ((T+P)/N tokens of K and V) hides under one ring step of attention;
+// pass-Q otherwise.
+cp_status cp_select_ring_variant(int64_t t, int64_t p, int32_t n_h, int32_t n_kv, int32_t d, int32_t n_ranks,
+                                 int32_t elem_bytes, double link_bytes_per_s, double step_attn_s,
+                                 cp_ring_variant* variant, int32_t* reason) {
+  if (!variant || t < 0 || p < 0 || t + p == 0 || n_h < 1 || n_kv < 1 || n_h % n_kv || d < 1 || n_ranks < 1 ||
+      elem_bytes < 1 || !(link_bytes_per_s > 0.0) || !(step_attn_s >= 0.0))
+    return CP_ERR_INVALID_ARG;
+  const double miss = static_cast<double>(t) / static_cast<double>(t + p);
+  const double threshold = 2.0 * static_cast<double>(n_kv) / static_cast<double>(n_h);
+  int32_t why = 0;
+  if (miss > threshold) {
+    why = 1;
+  } else {
+    const double hop_bytes = static_cast<double>(t + p) / n_ranks * n_kv * d * 2.0 * elem_bytes;
+    if (hop_bytes / link_bytes_per_s <= step_attn_s) why = 2;
+  }
+  *variant = why ? CP_PASS_KV : CP_PASS_Q;
+  if (reason) *reason = why;
+  return CP_OK;
+}
+
 }  // extern "C"

@@ -154,6 +154,22 @@ cp_status cp_ring_comm_volume(const cp_range* ranges, const cp_block* blocks, in
                               cp_ring_variant variant, int32_t n_h, int32_t n_kv, int32_t d,
                               int64_t* hop_elems, int64_t* total, int64_t* all_to_all);
 
+/* Ring variant by Algorithm 1 (method page, section 3, "Pass-KV vs Pass-Q"):
+ *  1. pass-KV if the KV-cache miss rate t/(t+p) is above 2*n_kv/n_h (12.5%
+ *     for 128 query heads on 8 KV heads);
+ *  2. else pass-KV if one ring hop's SendRecv of a KV shard, (t+p)/n_ranks
+ *     tokens of K and V at elem_bytes each, over link_bytes_per_s, takes no
+ *     longer than step_attn_s, the caller's time for one ring step of
+ *     attention (so the transfer hides under compute);
+ *  3. else pass-Q.
+ * t: new tokens, p: cached tokens (t+p > 0). Writes the variant and the
+ * condition that chose pass-KV (1 or 2; 0 for pass-Q) to *reason (may be NULL).
+ * CP_ERR_INVALID_ARG on a negative size, n_h % n_kv != 0, a non-positive link
+ * bandwidth or a negative step time. Host only. */
+cp_status cp_select_ring_variant(int64_t t, int64_t p, int32_t n_h, int32_t n_kv, int32_t d, int32_t n_ranks,
+                                 int32_t elem_bytes, double link_bytes_per_s, double step_attn_s,
+                                 cp_ring_variant* variant, int32_t* reason);
+
 /* ---------------------------------------------------------------------------
  * Device entry points (sm_100a). Pointers named q/k/v/o/lse/out/workspace are
  * device pointers; ranges/blocks are host arrays read during the call.

@@ -46,6 +46,27 @@ def select_variant(t: int, p: int, n_h: int, n_kv: int) -> int:
     return PASS_KV if t / (t + p) > miss_rate_threshold(n_h, n_kv) else PASS_Q
 
 
+def kv_hop_seconds(t: int, p: int, n_kv: int, d: int, n_ranks: int, elem_bytes: int,
+                   link_bytes_per_s: float) -> float:
+    """Time of one pass-KV ring hop: one rank's KV shard, (T+P)/N tokens of K
+    and of V, over a link of the given bandwidth."""
+    return (t + p) / n_ranks * n_kv * d * 2 * elem_bytes / link_bytes_per_s
+
+
+def select_variant_alg1(t: int, p: int, n_h: int, n_kv: int, d: int, n_ranks: int, elem_bytes: int,
+                        link_bytes_per_s: float, step_attn_s: float):
+    """Algorithm 1 of the method page (section 3), both conditions, in order:
+    1. pass-KV if the miss rate T/(T+P) is above 2*N_KV/N_H;
+    2. pass-KV if one ring hop's SendRecv of a KV shard takes no longer than
+       one ring step of attention (step_attn_s), i.e. it hides under compute;
+    otherwise pass-Q. Returns (variant, condition that chose pass-KV or 0)."""
+    if t / (t + p) > miss_rate_threshold(n_h, n_kv):
+        return PASS_KV, 1
+    if kv_hop_seconds(t, p, n_kv, d, n_ranks, elem_bytes, link_bytes_per_s) <= step_attn_s:
+        return PASS_KV, 2
+    return PASS_Q, 0
+
+
 def schedule_volume(ranges, blocks, n_ranks: int, variant: int, n_h: int, n_kv: int, d: int):
     """Per hop and per rank, the elements a rank receives (per tensor for
     pass-KV; the Q tensor for pass-Q), plus pass-Q's all-to-all of (O, LSE).

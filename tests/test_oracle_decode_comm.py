@@ -100,3 +100,28 @@ def test_pass_q_volume():
     vol = C.schedule_volume(ranges, blocks, n, P.PASS_Q, n_h, 8, d)
     assert vol["total"] == (n - 1) * t * n_h * d
     assert vol["all_to_all"] == (n - 1) * t * n_h * (d + 1)
+
+
+def test_algorithm1_second_condition():
+    """Condition 2 of Algorithm 1: below the miss-rate threshold pass-KV is
+    still chosen when one KV hop hides under one ring step of attention. Pins:
+    the hop time of the page's switch point (T=6400, P=121600, 8 KV heads of
+    128, 8 ranks, bf16) is 16000 tokens x 8 x 128 x 2 tensors x 2 bytes =
+    65,536,000 bytes over the link; the conditions apply in order."""
+    n_h, n_kv, d, n, eb = 128, 8, 128, 8, 2
+    t, p = 6400, 121600
+    link = 50e9   # 400 Gb/s per GPU, the page's RDMA network
+    hop = C.kv_hop_seconds(t, p, n_kv, d, n, eb, link)
+    assert hop == 65_536_000 / link
+    assert C.select_variant_alg1(t, p, n_h, n_kv, d, n, eb, link, hop) == (P.PASS_KV, 2)          # hides exactly
+    assert C.select_variant_alg1(t, p, n_h, n_kv, d, n, eb, link, hop * 0.999) == (P.PASS_Q, 0)   # does not
+    # condition 1 wins regardless of timing
+    assert C.select_variant_alg1(64000, 64000, n_h, n_kv, d, n, eb, link, 0.0) == (P.PASS_KV, 1)
+    # at exactly the threshold condition 1 does not fire (strict), condition 2 decides
+    assert C.select_variant_alg1(16000, 112000, n_h, n_kv, d, n, eb, link, 0.0) == (P.PASS_Q, 0)
+    # a faster link turns the same workload to pass-KV
+    assert C.select_variant_alg1(t, p, n_h, n_kv, d, n, eb, 770e9, hop / 10)[0] == P.PASS_KV
+    # with condition 2 unsatisfiable, the choice is condition 1 alone
+    for tt in range(100, 128000, 3100):
+        assert C.select_variant_alg1(tt, 128000 - tt, n_h, n_kv, d, n, eb, link, 0.0)[0] == \
+            C.select_variant(tt, 128000 - tt, n_h, n_kv)

@@ -153,3 +153,21 @@ def test_decode_shards_partition_every_request(n_ranks, mode):
             assert np.all((rows >= offsets[b]) & (rows < offsets[b + 1]))
             seen[rows] += 1
     assert np.all(seen == 1)
+
+
+def test_select_ring_variant_matches_oracle():
+    """The library's Algorithm 1 equals the oracle's on a grid of miss rates,
+    head counts, rank counts, link speeds and step times."""
+    total = 128000
+    for n_h, n_kv in ((128, 8), (16, 1), (32, 8)):
+        for n in (2, 8):
+            for link in (12.5e9, 50e9, 770e9):
+                for step in (0.0, 1e-4, 1e-3, 1e-2):
+                    for t in (1, 1280, 6400, 16000, 16001, 40000, 127999):
+                        want = OC.select_variant_alg1(t, total - t, n_h, n_kv, 128, n, 2, link, step)
+                        got = B.cp_select_ring_variant(t, total - t, n_h, n_kv, 128, n, 2, link, step)
+                        assert got == want, (n_h, n_kv, n, link, step, t)
+    with pytest.raises(B.CpError):
+        B.cp_select_ring_variant(0, 0, 128, 8, 128, 8, 2, 50e9, 0.0)
+    with pytest.raises(B.CpError):
+        B.cp_select_ring_variant(10, 10, 128, 8, 128, 8, 2, 0.0, 0.0)
