@@ -43,7 +43,7 @@ EXPORTED = (
     "cp_status_string", "cp_abi_version", "cp_shard_plan", "cp_rank_ranges", "cp_ring_schedule",
     "cp_classify_pair", "cp_block_pairs", "cp_ring_comm_volume", "cp_workspace_size",
     "cp_reset_status", "cp_check_status", "cp_attn_partial", "cp_attn_merge", "cp_decode",
-    "cp_decode_static", "cp_decode_partial", "cp_select_ring_variant",
+    "cp_decode_static", "cp_decode_partial", "cp_select_ring_variant", "cp_attn_partial_fused",
 )
 
 
@@ -96,6 +96,8 @@ def lib() -> ctypes.CDLL:
         "cp_check_status": (i32, [vp, vp]),
         "cp_attn_partial": (i32, [vp, vp, vp, i32, i64, i64, i32, i32, i32, f32, i32, P(cp_range), i32,
                                   P(cp_block), i32, vp, vp, i64, vp, sz, vp]),
+        "cp_attn_partial_fused": (i32, [vp, vp, vp, i32, i64, i64, i32, i32, i32, f32, i32, P(cp_range), i32,
+                                        P(cp_block), i32, vp, vp, i64, i32, vp, vp, sz, vp]),
         "cp_attn_merge": (i32, [vp, vp, i32, i64, i64, i32, i32, vp, i32, vp, vp]),
         "cp_decode": (i32, [vp, vp, vp, i32, vp, i32, i64, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]),
         "cp_decode_static": (i32, [vp, vp, vp, i32, vp, i32, i64, i32, i32, i32, i32, f32, vp, vp, vp]),
@@ -239,6 +241,20 @@ def cp_attn_partial(q, k, v, n_h: int, n_kv: int, softmax_scale: float, causal: 
                                  n_blocks, _ptr(o_part), _ptr(lse_part), int(o_part.shape[0]), _ptr(workspace),
                                  int(workspace.numel() * workspace.element_size()), _stream(stream))
     _check("cp_attn_partial", code)
+
+
+def cp_attn_partial_fused(q, k, v, n_h: int, n_kv: int, softmax_scale: float, causal: bool, ranges, n_ranges: int,
+                          blocks, n_blocks: int, o_acc, lse_acc, accumulate: bool, out=None, workspace=None,
+                          stream=None) -> None:
+    """cp_attn_partial merging into the running (o_acc, lse_acc) when `accumulate`;
+    with `out` (bf16 [rows, n_h, d]) the merged rows are written there normalised."""
+    d = int(q.shape[-1])
+    code = lib().cp_attn_partial_fused(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), int(q.shape[0]), int(k.shape[0]),
+                                       n_h, n_kv, d, float(softmax_scale), int(causal), ranges, n_ranges, blocks,
+                                       n_blocks, _ptr(o_acc), _ptr(lse_acc), int(o_acc.shape[0]), int(bool(accumulate)),
+                                       _ptr(out), _ptr(workspace), int(workspace.numel() * workspace.element_size()),
+                                       _stream(stream))
+    _check("cp_attn_partial_fused", code)
 
 
 def cp_attn_merge(o_parts, lse_parts, n_parts: int, part_stride_rows: int, rows: int, n_h: int, d: int, out,

@@ -244,13 +244,16 @@ cp_status cp_check_status(const void* workspace, void* cuda_stream) {
   return CP_OK;
 }
 
-cp_status cp_attn_partial(const void* q, const void* k, const void* v, cp_dtype dtype, int64_t q_rows,
-                          int64_t kv_rows, int32_t n_h, int32_t n_kv, int32_t d, float softmax_scale, int32_t causal,
-                          const cp_range* ranges, int32_t n_ranges, const cp_block* blocks, int32_t n_blocks,
-                          float* o_part, float* lse_part, int64_t out_rows, void* workspace, size_t ws_bytes,
-                          void* cuda_stream) {
+static cp_status partial_impl(const void* q, const void* k, const void* v, cp_dtype dtype, int64_t q_rows,
+                              int64_t kv_rows, int32_t n_h, int32_t n_kv, int32_t d, float softmax_scale,
+                              int32_t causal, const cp_range* ranges, int32_t n_ranges, const cp_block* blocks,
+                              int32_t n_blocks, float* o_part, float* lse_part, int64_t out_rows, int32_t accumulate,
+                              void* out_final, void* workspace, size_t ws_bytes, void* cuda_stream) {
   // ---- arguments
   if (!q || !k || !v || !o_part || !lse_part) return CP_ERR_INVALID_ARG;
+  const bool fused = accumulate != 0 || out_final != nullptr;
+  if (fused && dtype != CP_BF16) return CP_ERR_UNSUPPORTED;
+  if (out_final && !aligned(out_final, 16)) return CP_ERR_INVALID_ARG;
   if (n_blocks < 0 || n_ranges < 0 || (n_blocks > 0 && (!ranges || !blocks))) return CP_ERR_INVALID_ARG;
   if (n_h < 1 || n_kv < 1 || d < 1 || q_rows < 0 || kv_rows < 0 || out_rows < 0) return CP_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.0f) || !(softmax_scale < INFINITY)) return CP_ERR_INVALID_ARG;
@@ -283,6 +286,18 @@ cp_status cp_attn_partial(const void* q, const void* k, const void* v, cp_dtype 
       if (!range_ok(r) || r.row0 + r.len > kv_rows) return CP_ERR_INVALID_ARG;
     }
   }
+  if (fused) {
+    // each output row may belong to at most one block of the call (read-modify-write)
+    std::vector<std::pair<int64_t, int64_t>> rows;
+    for (int32_t b = 0; b < n_blocks; ++b)
+      for (int32_t j = 0; j < blocks[b].q_count; ++j) {
+        const cp_range& r = ranges[blocks[b].q_begin + j];
+        if (r.len > 0) rows.emplace_back(blocks[b].out_row0 + r.row0, blocks[b].out_row0 + r.row0 + r.len);
+      }
+    std::sort(rows.begin(), rows.end());
+    for (size_t i = 1; i < rows.size(); ++i)
+      if (rows[i].first < rows[i - 1].second) return CP_ERR_INVALID_ARG;
+  }
   // tokens per CTA tile: the tensor-core kernel takes two 128-row query tiles per CTA
   const int tok_per_tile = (dtype == CP_BF16) ? tc::kQTiles * (128 / group) : simt::kRows / group;
   std::vector<WorkTable> tables;
@@ -303,6 +318,8 @@ cp_status cp_attn_partial(const void* q, const void* k, const void* v, cp_dtype 
     if (!make_qkv_maps(params, q, k, v, q_rows, kv_rows, n_h, n_kv, group)) return CP_ERR_CUDA;
     params.o_part = o_part;
     params.lse_part = lse_part;
+    params.out_final = static_cast<__nv_bfloat16*>(out_final);
+    params.accumulate = accumulate != 0;
     params.status = status;
     params.n_h = n_h;
     params.log2_group = ilog2_exact(group);
@@ -345,6 +362,24 @@ cp_status cp_attn_partial(const void* q, const void* k, const void* v, cp_dtype 
     }
   }
   return CP_OK;
+}
+
+cp_status cp_attn_partial(const void* q, const void* k, const void* v, cp_dtype dtype, int64_t q_rows,
+                          int64_t kv_rows, int32_t n_h, int32_t n_kv, int32_t d, float softmax_scale, int32_t causal,
+                          const cp_range* ranges, int32_t n_ranges, const cp_block* blocks, int32_t n_blocks,
+                          float* o_part, float* lse_part, int64_t out_rows, void* workspace, size_t ws_bytes,
+                          void* cuda_stream) {
+  return partial_impl(q, k, v, dtype, q_rows, kv_rows, n_h, n_kv, d, softmax_scale, causal, ranges, n_ranges, blocks,
+                      n_blocks, o_part, lse_part, out_rows, 0, nullptr, workspace, ws_bytes, cuda_stream);
+}
+
+cp_status cp_attn_partial_fused(const void* q, const void* k, const void* v, cp_dtype dtype, int64_t q_rows,
+                                int64_t kv_rows, int32_t n_h, int32_t n_kv, int32_t d, float softmax_scale,
+                                int32_t causal, const cp_range* ranges, int32_t n_ranges, const cp_block* blocks,
+                                int32_t n_blocks, float* o_acc, float* lse_acc, int64_t out_rows, int32_t accumulate,
+                                void* out, void* workspace, size_t ws_bytes, void* cuda_stream) {
+  return partial_impl(q, k, v, dtype, q_rows, kv_rows, n_h, n_kv, d, softmax_scale, causal, ranges, n_ranges, blocks,
+                      n_blocks, o_acc, lse_acc, out_rows, accumulate, out, workspace, ws_bytes, cuda_stream);
 }
 
 cp_status cp_attn_merge(const float* o_parts, const float* lse_parts, int32_t n_parts, int64_t part_stride_rows,

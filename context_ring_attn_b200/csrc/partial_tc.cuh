@@ -91,6 +91,8 @@ struct Params {
   CUtensorMap tm_v;
   float* o_part;
   float* lse_part;
+  __nv_bfloat16* out_final;   // not null: write the merged, normalised row here (bf16) instead of o_part
+  int32_t accumulate;         // merge each row into the (O, LSE) already at its place in o_part / lse_part
   uint32_t* status;
   int32_t n_h;
   int32_t log2_group;
@@ -437,41 +439,80 @@ __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Para
     }
 
     // ---------------------------------------------------------------- epilogue
+    // This block's row: O_blk = O / l and LSE_blk = m + ln l. Written as is, or
+    // (accumulate) merged into the row's earlier (O, LSE) by LSE weighting
+    // ("merge attention", method page section 5): M = max(LSE_prev, LSE_blk),
+    // w = exp(LSE - M), O = (w_prev O_prev + w_blk O_blk) / (w_prev + w_blk),
+    // LSE = M + ln(w_prev + w_blk); a part at -inf weighs 0.
     const int64_t out_row = ws.out_row0 + q_row0 + tok;
     const int head = kvh * group + (row & (group - 1));
+    const int64_t out_idx = out_row * p.n_h + head;
     bool done_ok = __all_sync(0xffffffffu, ok);
     if (done_ok && n_iter > 0) done_ok = warp_wait(&bars[B_O_DONE + x], (n_iter - 1) & 1, abort_flag, p.status);
+    // both halves read the earlier LSE before either may overwrite it (after the barrier)
+    const float lse_prev = (p.accumulate && row_valid) ? p.lse_part[out_idx] : -INFINITY;
     // Whole row sum from the two halves. The partner warps agree on the
     // outcome here as in the loop (both reach this barrier exactly once).
     *xch_mine = l_run;
     done_ok = named_bar_and(pair_bar, 64, done_ok);
     const float l_tot = l_run + *xch_peer;
-    float* dst = p.o_part + (out_row * p.n_h + head) * HD + hf * 64;
-    if (done_ok && n_iter > 0) {
-      tc_fence_after();
-      const float inv_l = (l_tot > 0.0f) ? 1.0f / l_tot : 0.0f;
+    const float inv_l = (l_tot > 0.0f) ? 1.0f / l_tot : 0.0f;
+    const float lse_blk = (n_iter > 0 && l_tot > 0.0f) ? (m_run + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
+    float wa = 0.0f, wb = inv_l, lse_new = lse_blk;   // row = wa * O_prev + wb * O (TMEM)
+    if (p.accumulate) {
+      const float mx = fmaxf(lse_prev, lse_blk);
+      if (mx == -INFINITY) {
+        wb = 0.0f;
+      } else {
+        const float ep = expf(lse_prev - mx), eb = expf(lse_blk - mx);
+        const float sum = ep + eb;
+        wa = ep / sum;
+        wb = eb / sum * inv_l;
+        lse_new = mx + logf(sum);
+      }
+    }
+    float* dst = p.o_part + out_idx * HD + hf * 64;
+    if (done_ok) {
+      if (n_iter > 0) tc_fence_after();
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t o[32];
-        tmem_ld32(o_col + c * 32, o);
-        tmem_ld_wait();
-        if (row_valid) {
+        if (n_iter > 0) {
+          tmem_ld32(o_col + c * 32, o);
+          tmem_ld_wait();
+        } else {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            float4 v4 = make_float4(__uint_as_float(o[i]) * inv_l, __uint_as_float(o[i + 1]) * inv_l,
-                                    __uint_as_float(o[i + 2]) * inv_l, __uint_as_float(o[i + 3]) * inv_l);
-            *reinterpret_cast<float4*>(dst + c * 32 + i) = v4;
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        if (row_valid) {
+          float r[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(o[i]) * wb;
+          if (p.accumulate) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 pv = *reinterpret_cast<const float4*>(dst + c * 32 + i);
+              r[i] = fmaf(wa, pv.x, r[i]);
+              r[i + 1] = fmaf(wa, pv.y, r[i + 1]);
+              r[i + 2] = fmaf(wa, pv.z, r[i + 2]);
+              r[i + 3] = fmaf(wa, pv.w, r[i + 3]);
+            }
+          }
+          if (p.out_final) {
+            uint4* fo = reinterpret_cast<uint4*>(p.out_final + out_idx * HD + hf * 64 + c * 32);
+#pragma unroll
+            for (int i = 0; i < 32; i += 8)
+              fo[i >> 3] = make_uint4(pack_bf16x2(r[i], r[i + 1]), pack_bf16x2(r[i + 2], r[i + 3]),
+                                      pack_bf16x2(r[i + 4], r[i + 5]), pack_bf16x2(r[i + 6], r[i + 7]));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(dst + c * 32 + i) = make_float4(r[i], r[i + 1], r[i + 2], r[i + 3]);
           }
         }
       }
-    } else if (done_ok && n_iter == 0 && row_valid) {
-#pragma unroll
-      for (int i = 0; i < 64; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if (done_ok && row_valid && hf == 0) {
-      const float lse = (l_tot > 0.0f) ? (m_run + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
-      p.lse_part[out_row * p.n_h + head] = lse;
-    }
+    if (done_ok && row_valid && hf == 0) p.lse_part[out_idx] = lse_new;
   }
 
   tc_fence_before();

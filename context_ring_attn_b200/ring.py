@@ -73,17 +73,28 @@ def run_ring(sched: RingSchedule, q, k, v, n_h: int, n_kv: int, out, lse_out=Non
     merge="final": N partial buffers, one N-way merge at the end.
     merge="running": two partial buffers; after every step the step's partial
     is merged into the running one (less memory, N-1 extra merge passes).
+    merge="fused": one buffer; every step's kernel merges its rows into the
+    running (O, LSE) in its epilogue and the last step writes `out` directly
+    (cp_attn_partial_fused; no merge pass). lse_out, if given, is the running
+    LSE buffer.
     """
     q_rows, d = int(q.shape[0]), int(q.shape[-1])
     n = sched.n_ranks
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    n_bufs = n if merge == "final" else 2
+    n_bufs = n if merge == "final" else (1 if merge == "fused" else 2)
     if o_parts is None:
         o_parts, lse_parts = partial_buffers(q_rows, n_h, d, n_bufs, q.device)
     if workspace is None:
         workspace = torch.zeros(B.cp_workspace_size(B.CP_OP_PARTIAL, 0, n_h, d, 1), dtype=torch.uint8,
                                 device=q.device)
+    if merge == "fused":
+        lse_acc = lse_out if lse_out is not None else lse_parts
+        for t in range(n):
+            blocks = sched.step_blocks(t, q_rows, part_of=lambda _p: 0)
+            B.cp_attn_partial_fused(q, k, v, n_h, n_kv, scale, causal, sched.ranges, sched.n_ranges, blocks, n,
+                                    o_parts, lse_acc, t > 0, out if t == n - 1 else None, workspace, stream)
+        return out
     if merge == "final":
         for t in range(n):
             blocks = sched.step_blocks(t, q_rows)

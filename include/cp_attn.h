@@ -216,6 +216,26 @@ cp_status cp_attn_partial(const void* q, const void* k, const void* v, cp_dtype 
                           float* o_part, float* lse_part, int64_t out_rows, void* workspace,
                           size_t ws_bytes, void* cuda_stream);
 
+/* cp_attn_partial with the LSE merge in its epilogue ("merge attention",
+ * method page section 5, fused into the attention kernel), so that a ring
+ * schedule keeps one running (O, LSE) and needs no separate merge pass.
+ * Arguments as cp_attn_partial, with o_acc / lse_acc in the roles of o_part /
+ * lse_part, and:
+ *   accumulate = 0: each computed row is written as cp_attn_partial writes it;
+ *   accumulate != 0: each computed row is merged into the (O, LSE) already at
+ *     its place in o_acc / lse_acc (LSE weighting; -inf weighs 0);
+ *   out (bf16 [out_rows, n_h, d], 16-byte aligned) not NULL: the resulting row
+ *     is written there normalised instead of to o_acc (lse_acc still gets its
+ *     LSE): the last step of a ring.
+ * A row written by this call must belong to one block only (the host checks
+ * this and returns CP_ERR_INVALID_ARG otherwise). dtype CP_BF16 only
+ * (CP_ERR_UNSUPPORTED for CP_F32). */
+cp_status cp_attn_partial_fused(const void* q, const void* k, const void* v, cp_dtype dtype, int64_t q_rows,
+                                int64_t kv_rows, int32_t n_h, int32_t n_kv, int32_t d, float softmax_scale,
+                                int32_t causal, const cp_range* ranges, int32_t n_ranges, const cp_block* blocks,
+                                int32_t n_blocks, float* o_acc, float* lse_acc, int64_t out_rows, int32_t accumulate,
+                                void* out, void* workspace, size_t ws_bytes, void* cuda_stream);
+
 /* LSE merge of n_parts partials of the same rows (method page, section 5,
  * implementation detail 3: the merge after pass-Q; the same step closes
  * pass-KV). Part j lives at o_parts + j*part_stride_rows*n_h*d and

@@ -275,3 +275,45 @@ def test_decode_replays_from_a_cuda_graph():
     B.cp_check_status(ws)
     o_ref2, l_ref2 = OD.decode(dc2.q, dc2.k, dc2.v, dc2.offsets)
     check(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref2, l_ref2, "bf16", "graph replay, new inputs")
+
+
+# ---------------------------------------------------------------------------- merge fused into the partial epilogue
+@pytest.mark.parametrize("t,n_h,n_kv,n_ranks,variant,p", [
+    (1000, 16, 1, 3, B.CP_PASS_KV, 0),
+    (777, 8, 2, 4, B.CP_PASS_Q, 0),
+    (300, 32, 2, 4, B.CP_PASS_Q, 1500),
+    (300, 16, 1, 1, B.CP_PASS_KV, 0),
+])
+def test_bf16_ring_fused_merge(t, n_h, n_kv, n_ranks, variant, p):
+    """The ring with the LSE merge in the partial kernel's epilogue (one running
+    buffer, the last step writes bf16 out) equals unsharded attention."""
+    pr = synth.make_prefill(t, n_h, n_kv, 128, "bf16", 200 + t, 0.5, p=p)
+    _run_prefill(pr, n_ranks, variant, B.CP_SHARD_LOAD_BALANCED, merge="fused")
+
+
+def test_bf16_varlen_fused_merge():
+    lens = [700, 129, 1000]
+    segs, r0 = [], 0
+    for i, n in enumerate(lens):
+        segs.append(ring.Segment(n, r0, 0, i))
+        r0 += n
+    pr = synth.make_prefill(sum(lens), 16, 2, 128, "bf16", 6, 0.5)
+    _run_prefill(pr, 3, B.CP_PASS_KV, B.CP_SHARD_LOAD_BALANCED, merge="fused", segs=segs)
+
+
+def test_fused_rejects_overlapping_rows_and_fp32():
+    rng = np.random.default_rng(8)
+    q = dev(synth.bf16_bits(rng.standard_normal((64, 16, 128)).astype(np.float32)), "bf16")
+    k = dev(synth.bf16_bits(rng.standard_normal((64, 1, 128)).astype(np.float32)), "bf16")
+    o = torch.zeros((64, 16, 128), device="cuda")
+    lse = torch.zeros((64, 16), device="cuda")
+    ranges = (B.cp_range * 2)(B.cp_range(0, 0, 64, 0, 0), B.cp_range(0, 0, 64, 0, 0))
+    blocks = (B.cp_block * 2)(B.cp_block(0, 1, 1, 1, 0), B.cp_block(0, 1, 1, 1, 0))   # same rows twice
+    with pytest.raises(B.CpError) as e:
+        B.cp_attn_partial_fused(q, k, k, 16, 1, 0.1, True, ranges, 2, blocks, 2, o, lse, True, None, _ws())
+    assert e.value.code == B.CP_ERR_INVALID_ARG
+    qf = torch.zeros((64, 16, 64), device="cuda")
+    kf = torch.zeros((64, 1, 64), device="cuda")
+    with pytest.raises(B.CpError) as e:
+        B.cp_attn_partial_fused(qf, kf, kf, 16, 1, 0.1, True, ranges, 2, blocks, 1, o, lse, True, None, _ws())
+    assert e.value.code == B.CP_ERR_UNSUPPORTED
