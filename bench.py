@@ -291,19 +291,21 @@ def run_ours(args, rank: int, world: int):
             B.cp_attn_partial_fused(q, k, v, n_h, n_kv, scale, True, sched.ranges, sched.n_ranges, blocks, n_ranks,
                                     o_acc, lse, s > 0, out if s == n_ranks - 1 else None, ws)
 
-    for _ in range(max(2, args.warmup)):
+    fused_ms = None
+    for _ in range(0 if args.no_fused else max(2, args.warmup)):
         fused_step()
     barrier()
     torch.cuda.synchronize()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(args.steps):
-        fused_step()
-    f1.record(stream)
-    torch.cuda.synchronize()
-    B.cp_check_status(ws)
-    fused_ms = f0.elapsed_time(f1) / args.steps
-    if world > 1:
+    if not args.no_fused:
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            fused_step()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        B.cp_check_status(ws)
+        fused_ms = f0.elapsed_time(f1) / args.steps
+    if world > 1 and fused_ms is not None:
         tt = torch.tensor([fused_ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         fused_ms = float(tt.item())
@@ -341,10 +343,10 @@ def run_ours(args, rank: int, world: int):
         "merge": {"ms_per_step": merge_ms / args.steps,
                   "gbs": merge_bytes / (merge_ms / args.steps * 1e-3) / 1e9,
                   "frac_hbm": merge_bytes / (merge_ms / args.steps * 1e-3) / 1e9 / float(peaks["hbm_gbs"])},
-        "fused_merge": {"value": world * step_flops / (fused_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                        "ms_per_step": fused_ms,
-                        "note": "same step, LSE merge in the partial kernel's epilogue (cp_attn_partial_fused): "
-                                "8 launches, one running buffer, no merge pass"},
+        "fused_merge": None if fused_ms is None else {
+            "value": world * step_flops / (fused_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": fused_ms,
+            "note": "same step, LSE merge in the partial kernel's epilogue (cp_attn_partial_fused): "
+                    "8 launches, one running buffer, no merge pass"},
         "e2e": e2e,
         "gpu_launches": args.steps * (n_ranks + 1),
         "clocks": clk,
@@ -731,6 +733,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-fused", action="store_true", help="skip timing the fused-merge variant of the step")
     ap.add_argument("--no-secondary", action="store_true", help="skip the persistent-KV and varlen workloads")
     ap.add_argument("--only-decode", action="store_true", help="time the split-KV decode workload alone")
     ap.add_argument("--sweep-miss-rate", action="store_true",

@@ -317,3 +317,34 @@ def test_fused_rejects_overlapping_rows_and_fp32():
     with pytest.raises(B.CpError) as e:
         B.cp_attn_partial_fused(qf, kf, kf, 16, 1, 0.1, True, ranges, 2, blocks, 1, o, lse, True, None, _ws())
     assert e.value.code == B.CP_ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------------------- degenerate shapes
+@pytest.mark.parametrize("t,n_ranks,variant,merge", [
+    (5, 4, B.CP_PASS_KV, "final"),     # 8 chunks for 5 tokens: most shards empty
+    (1, 2, B.CP_PASS_Q, "final"),      # one token
+    (3, 8, B.CP_PASS_KV, "fused"),
+    (7, 3, B.CP_PASS_Q, "running"),
+])
+def test_bf16_ring_fewer_tokens_than_chunks(t, n_ranks, variant, merge):
+    pr = synth.make_prefill(t, 16, 1, 128, "bf16", 300 + t, 0.5)
+    _run_prefill(pr, n_ranks, variant, B.CP_SHARD_LOAD_BALANCED, merge=merge)
+
+
+def test_fp32_ring_fewer_tokens_than_chunks():
+    pr = synth.make_prefill(3, 4, 1, 64, "f32", 9, 1.0)
+    _run_prefill(pr, 4, B.CP_PASS_KV, B.CP_SHARD_LOAD_BALANCED)
+
+
+def test_decode_all_requests_empty():
+    lens = [0, 0, 0]
+    dc = synth.make_decode(len(lens), 16, 1, 128, lens, 90, 0.5)
+    q = dev(dc.q_raw, "bf16")
+    k = torch.zeros((1, 1, 128), dtype=torch.bfloat16, device="cuda")
+    off = torch.from_numpy(dc.offsets).cuda()
+    out = torch.full((3, 16, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((3, 16), float("nan"), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(B.cp_workspace_size(B.CP_OP_DECODE, 3, 16, 128, 8), dtype=torch.uint8, device="cuda")
+    B.cp_decode(q, k, k, off, 16, 1, 8, 1 / math.sqrt(128), out, lse, ws)
+    B.cp_check_status(ws)
+    assert torch.all(out.float() == 0) and torch.all(torch.isneginf(lse))
