@@ -120,38 +120,49 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint3
   }
 }
 
-// Exponentials of one half row (64 keys) for one KV tile: P = 2^(S*scale*log2e - m)
-// as bf16 pairs over the first 32 of the half row's S columns, returning the
-// sum of the fp32 values. The S half is read again from TMEM 16 columns at a
-// time, the next chunk in flight while this one is exponentiated (P chunk h8,
-// columns 8h8.., lies below every S chunk not yet read). kPolyPairsPer8 of
-// every 8 pairs take the polynomial on the FMA pipe, the rest the special
-// function unit. kMasked: keys past `lim` are hidden and get exactly 0 (the
-// polynomial or a large unmasked S would leave a value there); a separate
-// instantiation keeps the compares out of the unmasked tiles.
+// Exponentials of one half row (64 keys) for one KV tile: P = 2^(S*scale*log2e
+// - m_use) as 32 bf16 pairs in registers (pk), returning the sum of the fp32
+// values; nothing is written, so S stays in TMEM for a redo. S is read from
+// TMEM 8 columns at a time, the next chunk in flight while this one is
+// exponentiated. kPolyPairsPer8 of every 8 pairs take the polynomial on the
+// FMA pipe, the rest the special function unit. kMasked: keys past `lim` are
+// hidden and get exactly 0 (the polynomial or a large unmasked S would leave a
+// value there); a separate instantiation keeps the compares out of the
+// unmasked tiles. x_max receives the largest exponent S*scale*log2e - m_use
+// over the visible keys.
 template <bool kMasked>
-__device__ __forceinline__ float half_row_exps(uint32_t s_col, float sl2, float m_use, int lim) {
+__device__ __forceinline__ float half_row_exps(uint32_t s_col, float sl2, float m_use, int lim, uint32_t (&pk)[32],
+                                               float& x_max) {
+  float xm0 = -INFINITY, xm1 = -INFINITY;
   const uint64_t sl2_2 = f2_pack(sl2, sl2);
   const uint64_t negm_2 = f2_pack(-m_use, -m_use);
   uint64_t acc[2] = {0ull, 0ull};
-  uint32_t sc[2][16];
-  tmem_ld16(s_col, sc[0]);
+  uint32_t sc[2][8];
+  tmem_ld8(s_col, sc[0]);
   tmem_ld_wait();
 #pragma unroll
-  for (int h8 = 0; h8 < 4; ++h8) {
-    if (h8 < 3) tmem_ld16(s_col + (h8 + 1) * 16, sc[(h8 + 1) & 1]);
-    const uint32_t (&sv)[16] = sc[h8 & 1];
-    uint32_t pk[8];
+  for (int h4 = 0; h4 < 8; ++h4) {
+    if (h4 < 7) tmem_ld8(s_col + (h4 + 1) * 8, sc[(h4 + 1) & 1]);
+    const uint32_t (&sv)[8] = sc[h4 & 1];
 #pragma unroll
-    for (int cc = 0; cc < 16; cc += 2) {
-      const int c = h8 * 16 + cc;
+    for (int cc = 0; cc < 8; cc += 2) {
+      const int c = h4 * 8 + cc;
       const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[cc]), __uint_as_float(sv[cc + 1])), sl2_2, negm_2);
+      float x0, x1;
+      f2_unpack(x2, x0, x1);
+      if (kMasked) {
+        const float v0 = (c > lim) ? -INFINITY : x0;
+        const float v1 = (c + 1 > lim) ? -INFINITY : x1;
+        if ((c >> 1) & 1) xm1 = fmax3(xm1, v0, v1);
+        else xm0 = fmax3(xm0, v0, v1);
+      } else {
+        if ((c >> 1) & 1) xm1 = fmax3(xm1, x0, x1);
+        else xm0 = fmax3(xm0, x0, x1);
+      }
       uint64_t p2;
       if (((c >> 1) & 7) < kPolyPairsPer8) {
         p2 = exp2_poly_x2(x2);
       } else {
-        float x0, x1;
-        f2_unpack(x2, x0, x1);
         p2 = f2_pack(ex2(x0), ex2(x1));
       }
       if (kMasked) {
@@ -163,15 +174,15 @@ __device__ __forceinline__ float half_row_exps(uint32_t s_col, float sl2, float 
       }
       float p0, p1;
       f2_unpack(p2, p0, p1);
-      pk[cc >> 1] = pack_bf16x2(p0, p1);
+      pk[c >> 1] = pack_bf16x2(p0, p1);
       acc[(c >> 1) & 1] = f2_add(acc[(c >> 1) & 1], p2);
     }
-    tmem_st8(s_col + h8 * 8, pk);
-    if (h8 < 3) tmem_ld_wait();
+    if (h4 < 7) tmem_ld_wait();
   }
   const uint64_t t = f2_add(acc[0], acc[1]);
   float lo, hi;
   f2_unpack(t, lo, hi);
+  x_max = fmaxf(xm0, xm1);
   return lo + hi;
 }
 
@@ -366,58 +377,82 @@ __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Para
         const int n_valid = static_cast<int>(min(static_cast<int64_t>(BN), nv - k0));
         // S_x(it) is in TMEM; this also means O_x += P_x(it-1) V has completed
         const bool got = warp_wait(&bars[B_S_FULL + x], it & 1, abort_flag, p.status);
-        uint32_t s[2][32];
-        float mx = -INFINITY;
         // key hf*64 + c of the tile is visible iff c <= lim
         int lim = 63;
+        if ((n_valid < BN) || (causal && kp0 + BN - 1 > qpos)) {
+          int64_t l64 = n_valid - 1;
+          if (causal && qpos - kp0 < l64) l64 = qpos - kp0;
+          l64 -= hf * 64;
+          lim = static_cast<int>(max(min(l64, static_cast<int64_t>(63)), static_cast<int64_t>(-1)));
+        }
+        const bool tile_masked = __any_sync(0xffffffffu, lim < 63);
+        // Optimistic step: exponentiate against the running max m_run and track
+        // the tile's largest exponent. The P written is final unless a row of
+        // either half grew its max by more than 2^kRescaleThreshold, or has no
+        // running max yet (a first visible tile), which both halves detect
+        // alike (the two threads of a row hold the same m_run); then both take
+        // the exact step below. The partners' row maxima (raw, log2 units) are
+        // exchanged through shared memory before the vote.
+        const bool first = __any_sync(0xffffffffu, m_run == -INFINITY);
+        float raw_max = -INFINITY;   // max over visible keys of S*scale*log2e in this half row
+        float sum = 0.0f;
+        bool fine = false;
+        uint32_t pk[32];             // P of this half row, bf16 pairs
         if (got) {
           tc_fence_after();
-          tmem_ld32(s_col, s[0]);
-          tmem_ld32(s_col + 32, s[1]);
-          tmem_ld_wait();
-          if ((n_valid < BN) || (causal && kp0 + BN - 1 > qpos)) {
-            int64_t l64 = n_valid - 1;
-            if (causal && qpos - kp0 < l64) l64 = qpos - kp0;
-            l64 -= hf * 64;
-            lim = static_cast<int>(max(min(l64, static_cast<int64_t>(63)), static_cast<int64_t>(-1)));
-          }
-          if (__any_sync(0xffffffffu, lim < 63)) {
+          if (first) {
+            float a0 = -INFINITY, a1 = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (c > lim) s[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-          }
-          float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+            for (int h16 = 0; h16 < 4; ++h16) {
+              uint32_t sv[16];
+              tmem_ld16(s_col + h16 * 16, sv);
+              tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 64; c += 8) {
-            a0 = fmax3(a0, __uint_as_float(s[c >> 5][(c + 0) & 31]), __uint_as_float(s[c >> 5][(c + 1) & 31]));
-            a1 = fmax3(a1, __uint_as_float(s[c >> 5][(c + 2) & 31]), __uint_as_float(s[c >> 5][(c + 3) & 31]));
-            a2 = fmax3(a2, __uint_as_float(s[c >> 5][(c + 4) & 31]), __uint_as_float(s[c >> 5][(c + 5) & 31]));
-            a3 = fmax3(a3, __uint_as_float(s[c >> 5][(c + 6) & 31]), __uint_as_float(s[c >> 5][(c + 7) & 31]));
+              for (int cc = 0; cc < 16; cc += 4) {
+                const int c = h16 * 16 + cc;
+                const float v0 = (c > lim) ? -INFINITY : __uint_as_float(sv[cc]);
+                const float v1 = (c + 1 > lim) ? -INFINITY : __uint_as_float(sv[cc + 1]);
+                const float v2 = (c + 2 > lim) ? -INFINITY : __uint_as_float(sv[cc + 2]);
+                const float v3 = (c + 3 > lim) ? -INFINITY : __uint_as_float(sv[cc + 3]);
+                a0 = fmax3(a0, v0, v1);
+                a1 = fmax3(a1, v2, v3);
+              }
+            }
+            raw_max = fmaxf(a0, a1) * sl2;
+          } else {
+            float x_max;
+            sum = tile_masked ? half_row_exps<true>(s_col, sl2, m_run, lim, pk, x_max)
+                              : half_row_exps<false>(s_col, sl2, m_run, lim, pk, x_max);
+            raw_max = x_max + m_run;
+            fine = !(x_max > kRescaleThreshold);
           }
-          mx = fmaxf(fmax3(a0, a1, a2), a3);
         }
-        // Row max across the two halves. Both warps always meet here once per
-        // KV tile and agree on whether to go on, so neither can wait alone.
-        // The peer reads this slot before it arrives on P_FULL, and the next
-        // write comes after S_FULL, which needs that arrival: no overwrite race.
-        *xch_mine = mx;
+        // Both warps of the pair always meet here once per KV tile and agree on
+        // the outcome, so neither can wait alone. The peer reads this slot
+        // before it arrives on P_FULL, and the next write comes after S_FULL,
+        // which needs that arrival: no overwrite race.
+        *xch_mine = raw_max;
         tc_fence_before();
-        if (!named_bar_and(pair_bar, 64, got)) { ok = false; break; }
+        const bool all_fine = named_bar_and(pair_bar, 64, got && fine);
         tc_fence_after();
-        mx = fmaxf(mx, *xch_peer);
-
-        const float m_new = fmaxf(m_run, mx * sl2);
         float alpha = 1.0f;
         bool resc = false;
-        if (m_new > m_run + kRescaleThreshold) {
-          alpha = ex2(m_run - m_new);
-          m_run = m_new;
-          resc = true;
+        if (!all_fine) {
+          if (!named_bar_and(pair_bar, 64, got)) { ok = false; break; }
+          // exact step: the row max over both halves; rescale if it grew past the threshold
+          const float m_new = fmaxf(m_run, fmaxf(raw_max, *xch_peer));
+          if (m_new > m_run + kRescaleThreshold) {
+            alpha = ex2(m_run - m_new);
+            m_run = m_new;
+            resc = true;
+          }
+          const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
+          float unused;
+          sum = tile_masked ? half_row_exps<true>(s_col, sl2, m_use, lim, pk, unused)
+                            : half_row_exps<false>(s_col, sl2, m_use, lim, pk, unused);
         }
-        const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
-        const bool tile_masked = __any_sync(0xffffffffu, lim < 63);
-        const float sum = tile_masked ? half_row_exps<true>(s_col, sl2, m_use, lim)
-                                      : half_row_exps<false>(s_col, sl2, m_use, lim);
+        // P over the first 32 columns of this half row's S (read by the PV MMA)
+        tmem_st32(s_col, pk);
         l_run = l_run * alpha + sum;
         // O_x holds every earlier PV (see S_FULL above): rescale this half in place if needed
         if (it > 0 && __any_sync(0xffffffffu, resc)) {
