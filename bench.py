@@ -317,6 +317,7 @@ def run_ours(args, rank: int, world: int):
     if not args.no_secondary:
         for name in ("persistent_kv", "varlen_prefill"):
             secondary[name] = run_secondary(args, dev, name)
+        secondary["varlen_prefill_running_merge"] = run_secondary(args, dev, "varlen_prefill", "running")
 
     if rank != 0:
         return
@@ -452,11 +453,13 @@ def run_e2e(args, q, k, v, out, lse, o_parts, lse_parts, ws, segs, n_ranks, n_h,
                     "neighbouring steps overlap the compute on two copy streams (double-buffered)"}
 
 
-def run_secondary(args, dev, name: str):
+def run_secondary(args, dev, name: str, merge_override: str | None = None):
     """The other prefill workloads, each a full ring schedule per step:
     persistent-KV partial prefill (T=4096 new over P=126976 cached, 128/8
     heads, pass-Q, 8-way merge) and the varlen batch (8 sequences, 262144
-    tokens, 128/8 heads, pass-KV, running 2-way merges to bound memory)."""
+    tokens, 128/8 heads, pass-KV, merge fused into the partial kernel: its
+    partials are 17 GB per part, so the ring keeps one running buffer;
+    merge_override="running" times separate 2-way merges instead)."""
     import torch
 
     from context_ring_attn_b200 import binding as B
@@ -476,12 +479,16 @@ def run_secondary(args, dev, name: str):
         t = w["total"]
         starts = np.concatenate([[0], np.cumsum(lens)[:-1]]).astype(np.int64)
         q_segs = kv_segs = [ring.Segment(int(ln), int(s0), 0, i) for i, (ln, s0) in enumerate(zip(lens, starts))]
-        kv_rows, variant, merge = t, B.CP_PASS_KV, "running"
-        desc = {"seq_lens": [int(x) for x in lens], "ring": "pass-KV", "merge": "running 2-way"}
+        kv_rows, variant, merge = t, B.CP_PASS_KV, "fused"
+        desc = {"seq_lens": [int(x) for x in lens], "ring": "pass-KV",
+                "merge": "fused into the partial kernel's epilogue (cp_attn_partial_fused), one running buffer"}
+    if merge_override == "running":
+        merge = "running"
+        desc["merge"] = "running 2-way (cp_attn_merge after every step)"
     q = synth.device_rows(w["seed"], synth.TENSOR_Q, t, (n_h, d), w["std"], "bf16", dev)
     k = synth.device_rows(w["seed"], synth.TENSOR_K, kv_rows, (n_kv, d), w["std"], "bf16", dev)
     v = synth.device_rows(w["seed"], synth.TENSOR_V, kv_rows, (n_kv, d), w["std"], "bf16", dev)
-    n_bufs = n if merge == "final" else 2
+    n_bufs = n if merge == "final" else (1 if merge == "fused" else 2)
     o_parts, lse_parts = ring.partial_buffers(t, n_h, d, n_bufs, dev)
     out = torch.empty((t, n_h, d), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((t, n_h), dtype=torch.float32, device=dev)
@@ -495,13 +502,22 @@ def run_secondary(args, dev, name: str):
     def step(record):
         sched = ring.RingSchedule(q_segs, kv_segs, n, variant)
         for s_ in range(n):
-            target = (lambda pt: pt) if merge == "final" else (lambda _pt, _t=(0 if s_ == 0 else 1): _t)
+            if merge == "final":
+                target = lambda pt: pt
+            elif merge == "fused":
+                target = lambda _pt: 0
+            else:
+                target = lambda _pt, _t=(0 if s_ == 0 else 1): _t
             blocks = sched.step_blocks(s_, t, part_of=target)
             e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) if record else None
             if e:
                 e[0].record(stream)
-            B.cp_attn_partial(q, k, v, n_h, n_kv, scale, True, sched.ranges, sched.n_ranges, blocks, n, o_parts,
-                              lse_parts, ws)
+            if merge == "fused":
+                B.cp_attn_partial_fused(q, k, v, n_h, n_kv, scale, True, sched.ranges, sched.n_ranges, blocks, n,
+                                        o_parts, lse, s_ > 0, out if s_ == n - 1 else None, ws)
+            else:
+                B.cp_attn_partial(q, k, v, n_h, n_kv, scale, True, sched.ranges, sched.n_ranges, blocks, n,
+                                  o_parts, lse_parts, ws)
             if e:
                 e[1].record(stream)
                 ev_part.append(e)
@@ -539,14 +555,15 @@ def run_secondary(args, dev, name: str):
     part_ms = sum(a.elapsed_time(b) for a, b in ev_part) / steps
     merge_ms = sum(a.elapsed_time(b) for (a, b), _ in ev_merge) / steps
     merge_bytes = sum(nb for _, nb in ev_merge) / steps
+    no_merge = merge_ms == 0
     peaks, kind = load_peaks()
     peak_t = float(peaks["bf16_tflops_sustained"])
     res = {"value": step_flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms, "steps": steps,
            "flops_per_step": step_flops, "N_H": n_h, "N_KV": n_kv, "cp_ranks": n, **desc,
            "partial_tflops": step_flops / (part_ms * 1e-3) / 1e12,
            "partial_frac": step_flops / (part_ms * 1e-3) / 1e12 / peak_t,
-           "merge_gbs": merge_bytes / (merge_ms * 1e-3) / 1e9,
-           "merge_frac_hbm": merge_bytes / (merge_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
+           "merge_gbs": None if no_merge else merge_bytes / (merge_ms * 1e-3) / 1e9,
+           "merge_frac_hbm": None if no_merge else merge_bytes / (merge_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
            "peak_kind": f"bf16_tflops_sustained / hbm_gbs ({kind})"}
     del q, k, v, o_parts, lse_parts, out, lse
     torch.cuda.empty_cache()
