@@ -49,7 +49,9 @@ def _chunk_edges(lengths, starts, n_ranks):
     return must
 
 
-def test_prefill_128k_pass_kv():
+@pytest.mark.parametrize("merge", ["final", "fused"])
+def test_prefill_128k_pass_kv(merge):
+    """The headline step (separate 8-way merge) and its fused-merge variant."""
     w = synth.WORKLOADS["prefill_128k"]
     t, n_h, n_kv, d, n = w["t"], w["n_h"], w["n_kv"], w["d"], w["n_ranks"]
     q, k, v = _dev(w, synth.TENSOR_Q, t, n_h), _dev(w, synth.TENSOR_K, t, n_kv), _dev(w, synth.TENSOR_V, t, n_kv)
@@ -58,7 +60,7 @@ def test_prefill_128k_pass_kv():
     out = torch.empty((t, n_h, d), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((t, n_h), dtype=torch.float32, device="cuda")
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
-    ring.run_ring(sched, q, k, v, n_h, n_kv, out, lse, workspace=ws)
+    ring.run_ring(sched, q, k, v, n_h, n_kv, out, lse, workspace=ws, merge=merge)
     B.cp_check_status(ws)
     rows = sample_rows(np.random.default_rng(2), t, 1024, _chunk_edges([t], [0], n))
     o_gpu = out[torch.from_numpy(rows).cuda()].float().cpu().numpy()
@@ -117,7 +119,10 @@ def test_decode_split_full():
     check(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "bf16", "decode_split")
 
 
-def test_varlen_prefill_pass_kv():
+@pytest.mark.parametrize("merge", ["fused", "running"])
+def test_varlen_prefill_pass_kv(merge):
+    """The full varlen workload in both merge modes the bench times (fused is
+    the workload's default)."""
     w = synth.WORKLOADS["varlen_prefill"]
     lens = synth.varlen_lengths(w["seed"], w["n_seq"], w["total"])
     total, n_h, n_kv, d, n = w["total"], w["n_h"], w["n_kv"], w["d"], w["n_ranks"]
@@ -129,7 +134,7 @@ def test_varlen_prefill_pass_kv():
     out = torch.empty((total, n_h, d), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((total, n_h), dtype=torch.float32, device="cuda")
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
-    ring.run_ring(sched, q, k, v, n_h, n_kv, out, lse, workspace=ws, merge="running")
+    ring.run_ring(sched, q, k, v, n_h, n_kv, out, lse, workspace=ws, merge=merge)
     B.cp_check_status(ws)
     must = [int(s) for s in starts] + [int(s + ln - 1) for s, ln in zip(starts, lens)]
     must += _chunk_edges([lens[0]], [0], n)
