@@ -348,3 +348,33 @@ def test_decode_all_requests_empty():
     B.cp_decode(q, k, k, off, 16, 1, 8, 1 / math.sqrt(128), out, lse, ws)
     B.cp_check_status(ws)
     assert torch.all(out.float() == 0) and torch.all(torch.isneginf(lse))
+
+
+# ---------------------------------------------------------------------------- running-max growth
+@pytest.mark.parametrize("c,variant", [(4.0, B.CP_PASS_KV), (12.0, B.CP_PASS_KV), (12.0, B.CP_PASS_Q),
+                                       (16.0, B.CP_PASS_KV)])
+def test_bf16_score_jumps(c, variant):
+    """Queries share a common direction and a few keys point along it with
+    growing magnitude, so a row's max jumps by about 8c log2 units between KV
+    tiles: c = 4 exercises the deferred move to a new reference (growth past
+    2^8), c >= 12 the repeated step (growth past 2^64)."""
+    rng = np.random.default_rng(int(c * 10) + variant)
+    t, n_h, n_kv, d = 1100, 16, 1, 128
+    q = (0.5 + 0.1 * rng.standard_normal((t, n_h, d))).astype(np.float32)
+    k = (0.5 * rng.standard_normal((t, n_kv, d))).astype(np.float32)
+    v = rng.standard_normal((t, n_kv, d)).astype(np.float32)
+    for pos, mult in ((300, 0.5), (650, 1.0), (900, 1.5)):
+        k[pos] = c * mult
+    q_raw, k_raw, v_raw = synth.bf16_bits(q), synth.bf16_bits(k), synth.bf16_bits(v)
+    qd, kd, vd = dev(q_raw, "bf16"), dev(k_raw, "bf16"), dev(v_raw, "bf16")
+    segs = [ring.Segment(t, 0, 0, 0)]
+    sched = ring.RingSchedule(segs, segs, 2, variant)
+    out = torch.empty((t, n_h, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((t, n_h), dtype=torch.float32, device="cuda")
+    ws = _ws()
+    ring.run_ring(sched, qd, kd, vd, n_h, n_kv, out, lse, workspace=ws)
+    torch.cuda.synchronize()
+    B.cp_check_status(ws)
+    qv, kv_, vv = (synth.bf16_bits_to_f32(x) for x in (q_raw, k_raw, v_raw))
+    o_ref, l_ref = OA.attention(qv, kv_, vv, np.arange(t), np.arange(t))
+    check(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "bf16", f"jumps c={c}")
