@@ -44,6 +44,7 @@ EXPORTED = (
     "cp_classify_pair", "cp_block_pairs", "cp_ring_comm_volume", "cp_workspace_size",
     "cp_reset_status", "cp_check_status", "cp_attn_partial", "cp_attn_merge", "cp_decode",
     "cp_decode_static", "cp_decode_partial", "cp_select_ring_variant", "cp_attn_partial_fused",
+    "cp_wait_selftest",
 )
 
 
@@ -96,6 +97,7 @@ def lib() -> ctypes.CDLL:
         "cp_check_status": (i32, [vp, vp]),
         "cp_attn_partial": (i32, [vp, vp, vp, i32, i64, i64, i32, i32, i32, f32, i32, P(cp_range), i32,
                                   P(cp_block), i32, vp, vp, i64, vp, sz, vp]),
+        "cp_wait_selftest": (i32, [vp, sz, ctypes.c_uint64, vp]),
         "cp_attn_partial_fused": (i32, [vp, vp, vp, i32, i64, i64, i32, i32, i32, f32, i32, P(cp_range), i32,
                                         P(cp_block), i32, vp, vp, i64, i32, vp, vp, sz, vp]),
         "cp_attn_merge": (i32, [vp, vp, i32, i64, i64, i32, i32, vp, i32, vp, vp]),
@@ -225,6 +227,13 @@ def cp_workspace_size(op: int, rows: int, n_h: int, d: int, n_splits: int) -> in
 
 def cp_reset_status(workspace, stream=None) -> None:
     _check("cp_reset_status", lib().cp_reset_status(_ptr(workspace), _stream(stream)))
+
+
+def cp_wait_selftest(workspace, budget_ns: int, stream=None) -> None:
+    """Launch the bounded-wait self-test: the status word of `workspace` then
+    holds a timeout (cp_check_status raises CP_ERR_TIMEOUT)."""
+    _check("cp_wait_selftest", lib().cp_wait_selftest(_ptr(workspace), int(workspace.numel() * workspace.element_size()),
+                                                      int(budget_ns), _stream(stream)))
 
 
 def cp_check_status(workspace, stream=None) -> None:

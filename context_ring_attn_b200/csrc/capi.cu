@@ -227,6 +227,28 @@ size_t cp_workspace_size(cp_op op, int64_t rows, int32_t n_h, int32_t d, int32_t
   return kStatusBytes;
 }
 
+namespace {
+// One thread waits on a barrier that nothing arrives at, through the same
+// bounded wait as every kernel of the library, with a short budget.
+__global__ void wait_selftest_kernel(uint32_t* status, uint64_t budget_ns) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x != 0) return;
+  cpk::mbar_init(&bar, 1u);
+  abort_flag = 0u;
+  cpk::fence_mbar_init();
+  (void)cpk::mbar_wait(&bar, 0u, &abort_flag, status, budget_ns);
+}
+}  // namespace
+
+cp_status cp_wait_selftest(void* workspace, size_t ws_bytes, uint64_t budget_ns, void* cuda_stream) {
+  if (!workspace || ws_bytes < kStatusBytes || !aligned(workspace, 256)) return CP_ERR_WORKSPACE;
+  if (budget_ns == 0 || budget_ns > cpk::kWaitBudgetNs) return CP_ERR_INVALID_ARG;
+  wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(cuda_stream)>>>(static_cast<uint32_t*>(workspace),
+                                                                              budget_ns);
+  return last_cuda_status();
+}
+
 cp_status cp_reset_status(void* workspace, void* cuda_stream) {
   if (!workspace) return CP_ERR_WORKSPACE;
   if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)

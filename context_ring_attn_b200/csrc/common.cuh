@@ -17,7 +17,7 @@ constexpr uint32_t kStatusInternal = 2u;
 
 // A device-side wait gives up after this long (ns of %globaltimer). Correct
 // waits in these kernels last microseconds.
-constexpr uint64_t kWaitBudgetNs = 4000000000ull;
+constexpr uint64_t kWaitBudgetNs = 1000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -80,13 +80,13 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parit
 // CTA-wide abort flag is raised or after kWaitBudgetNs; on a timeout it raises
 // the abort flag and records kStatusTimeout in the status word.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag,
-                                          uint32_t* status) {
+                                          uint32_t* status, uint64_t budget_ns = kWaitBudgetNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
     if (*abort_flag) return false;
-    if (globaltimer() - t0 > kWaitBudgetNs) {
+    if (globaltimer() - t0 > budget_ns) {
       *abort_flag = 1u;
       if (status) atomicOr(status, kStatusTimeout);
       return false;

@@ -182,6 +182,15 @@ cp_status cp_select_ring_variant(int64_t t, int64_t p, int32_t n_h, int32_t n_kv
  *  cp_decode uses on any device. `rows` is the batch for decode. */
 size_t cp_workspace_size(cp_op op, int64_t rows, int32_t n_h, int32_t d, int32_t n_splits);
 
+/* Self-test of the library's device-side wait bound (no counterpart on the
+ * method's pages): one GPU thread waits on a barrier that nothing completes,
+ * through the same bounded wait every kernel uses, gives up after budget_ns
+ * (1 .. 1e9 ns; every other wait in the library gives up after 1 s) and
+ * records the timeout in the workspace status word, so that cp_check_status
+ * then returns CP_ERR_TIMEOUT. Nothing faults or hangs; the context stays
+ * usable. Asynchronous on the stream. */
+cp_status cp_wait_selftest(void* workspace, size_t ws_bytes, uint64_t budget_ns, void* cuda_stream);
+
 /* Zero the status word of a workspace (stream-ordered). */
 cp_status cp_reset_status(void* workspace, void* cuda_stream);
 

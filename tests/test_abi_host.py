@@ -138,3 +138,11 @@ def test_planning_rejects_bad_arguments(L):
         B.CP_ERR_INVALID_ARG   # needs 8 ranges, capacity 2
     assert L.cp_ring_schedule(segs, 1, segs, 1, 2, 0, 3, ranges, 2, ctypes.byref(n), blocks, None) == \
         B.CP_ERR_INVALID_ARG
+
+
+def test_wait_selftest_rejects_bad_arguments(L):
+    """Checked on the host before any launch."""
+    assert L.cp_wait_selftest(None, 256, 1000, None) == B.CP_ERR_WORKSPACE
+    assert L.cp_wait_selftest(FAKE, 128, 1000, None) == B.CP_ERR_WORKSPACE
+    assert L.cp_wait_selftest(FAKE, 256, 0, None) == B.CP_ERR_INVALID_ARG
+    assert L.cp_wait_selftest(FAKE, 256, 2_000_000_000, None) == B.CP_ERR_INVALID_ARG

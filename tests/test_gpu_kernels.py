@@ -378,3 +378,27 @@ def test_bf16_score_jumps(c, variant):
     qv, kv_, vv = (synth.bf16_bits_to_f32(x) for x in (q_raw, k_raw, v_raw))
     o_ref, l_ref = OA.attention(qv, kv_, vv, np.arange(t), np.arange(t))
     check(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "bf16", f"jumps c={c}")
+
+
+# ---------------------------------------------------------------------------- bounded waits
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A device-side wait on a barrier nothing completes gives up after its
+    budget and records CP_ERR_TIMEOUT; nothing faults, and the same context
+    then runs a decode correctly."""
+    ws = _ws()
+    B.cp_wait_selftest(ws, 20_000_000)   # 20 ms
+    torch.cuda.synchronize()
+    with pytest.raises(B.CpError) as e:
+        B.cp_check_status(ws)
+    assert e.value.code == B.CP_ERR_TIMEOUT
+    B.cp_reset_status(ws)
+    B.cp_check_status(ws)
+    lens = [100, 37]
+    dc, q, k, v, off = _decode_case(lens, 16, 1, 95)
+    out = torch.empty((2, 16, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((2, 16), dtype=torch.float32, device="cuda")
+    dws = torch.zeros(B.cp_workspace_size(B.CP_OP_DECODE, 2, 16, 128, 4), dtype=torch.uint8, device="cuda")
+    B.cp_decode(q, k, v, off, 16, 1, 4, 1 / math.sqrt(128), out, lse, dws)
+    B.cp_check_status(dws)
+    o_ref, l_ref = OD.decode(dc.q, dc.k, dc.v, dc.offsets)
+    check(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "bf16", "after timeout")
