@@ -402,3 +402,54 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     B.cp_check_status(dws)
     o_ref, l_ref = OD.decode(dc.q, dc.k, dc.v, dc.offsets)
     check(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "bf16", "after timeout")
+
+
+# ---------------------------------------------------------------------------- canaries after the outputs
+GUARD = 96   # rows of NaN after every output; no kernel may touch them
+
+
+def _guarded(shape, dtype):
+    t = torch.full((shape[0] + GUARD,) + tuple(shape[1:]), float("nan"), dtype=dtype, device="cuda")
+    return t, t[:shape[0]]
+
+
+def _guard_intact(t, rows):
+    return bool(torch.isnan(t[rows:].float()).all())
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_outputs_leave_guard_rows_untouched(dtype):
+    t, n_h, n_kv, d = 700, 16, 2, (128 if dtype == "bf16" else 64)
+    pr = synth.make_prefill(t, n_h, n_kv, d, dtype, 500, 0.5)
+    q_raw = pr.q_raw if dtype == "bf16" else pr.q.astype(np.float32)
+    q, k, v = dev(q_raw, dtype), dev(pr.k_raw, dtype), dev(pr.v_raw, dtype)
+    segs = [ring.Segment(t, 0, 0, 0)]
+    sched = ring.RingSchedule(segs, segs, 3, B.CP_PASS_KV)
+    o_full, o_parts = _guarded((3 * t, n_h, d), torch.float32)
+    l_full, l_parts = _guarded((3 * t, n_h), torch.float32)
+    out_dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    out_full, out = _guarded((t, n_h, d), out_dt)
+    lse_full, lse = _guarded((t, n_h), torch.float32)
+    ws = _ws()
+    ring.run_ring(sched, q, k, v, n_h, n_kv, out, lse, o_parts=o_parts, lse_parts=l_parts, workspace=ws)
+    torch.cuda.synchronize()
+    B.cp_check_status(ws)
+    for full, rows in ((o_full, 3 * t), (l_full, 3 * t), (out_full, t), (lse_full, t)):
+        assert _guard_intact(full, rows)
+    assert torch.isfinite(out.float()).all()
+
+
+def test_decode_leaves_guard_rows_untouched():
+    lens = [0, 300, 5000, 77]
+    dc, q, k, v, off = _decode_case(lens, 16, 1, 97)
+    out_full, out = _guarded((4, 16, 128), torch.bfloat16)
+    lse_full, lse = _guarded((4, 16), torch.float32)
+    o_full, o_part = _guarded((4, 16, 128), torch.float32)
+    lp_full, l_part = _guarded((4, 16), torch.float32)
+    ws = torch.zeros(B.cp_workspace_size(B.CP_OP_DECODE, 4, 16, 128, 64), dtype=torch.uint8, device="cuda")
+    B.cp_decode(q, k, v, off, 16, 1, 64, 1 / math.sqrt(128), out, lse, ws)
+    B.cp_decode_partial(q, k, v, off, 16, 1, 64, 1 / math.sqrt(128), o_part, l_part, ws)
+    torch.cuda.synchronize()
+    B.cp_check_status(ws)
+    for full, rows in ((out_full, 4), (lse_full, 4), (o_full, 4), (lp_full, 4)):
+        assert _guard_intact(full, rows)
