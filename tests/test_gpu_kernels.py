@@ -453,3 +453,14 @@ def test_decode_leaves_guard_rows_untouched():
     B.cp_check_status(ws)
     for full, rows in ((out_full, 4), (lse_full, 4), (o_full, 4), (lp_full, 4)):
         assert _guard_intact(full, rows)
+
+
+@pytest.mark.parametrize("t,n_h,n_kv,variant", [
+    (301, 32, 1, B.CP_PASS_KV),     # G = 32: 8 tokens per CTA tile
+    (129, 64, 1, B.CP_PASS_Q),      # G = 64
+    (77, 128, 1, B.CP_PASS_KV),     # G = 128: 2 tokens per CTA, one row per (token, head)
+    (150, 128, 2, B.CP_PASS_Q),     # G = 64 on two KV heads
+])
+def test_bf16_ring_large_gqa_groups(t, n_h, n_kv, variant):
+    pr = synth.make_prefill(t, n_h, n_kv, 128, "bf16", 600 + t, 0.5)
+    _run_prefill(pr, 2, variant, B.CP_SHARD_LOAD_BALANCED)
