@@ -14,6 +14,7 @@
 #include "merge.cuh"
 #include "partial_simt.cuh"
 #include "partial_tc.cuh"
+#include "partial_tc2.cuh"
 #include "work.cuh"
 
 namespace {
@@ -161,8 +162,10 @@ bool build_tables(const cp_range* ranges, const cp_block* blocks, int32_t n_bloc
 
 // Tensor maps: Q as [rows][N_KV][G][D] (box 64 x G x 1 x 128/G), K and V as
 // [rows][N_KV][D] (box 64 x 1 x 128), bf16, 128-byte swizzle.
-bool make_qkv_maps(tc::Params& p, const void* q, const void* k, const void* v, int64_t q_rows, int64_t kv_rows,
-                   int n_h, int n_kv, int group) {
+// Q box: 128 packed rows (128/G tokens x G heads) x 64 columns; K box: k_box_rows keys x 64 columns; V box:
+// 128 keys x 64 columns; 128-byte swizzle.
+bool make_qkv_maps(CUtensorMap* tm_q, CUtensorMap* tm_k, CUtensorMap* tm_v, const void* q, const void* k,
+                   const void* v, int64_t q_rows, int64_t kv_rows, int n_h, int n_kv, int group, int k_box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint32_t estr4[4] = {1, 1, 1, 1};
@@ -172,17 +175,17 @@ bool make_qkv_maps(tc::Params& p, const void* q, const void* k, const void* v, i
     const cuuint64_t strides[3] = {128 * 2, static_cast<cuuint64_t>(group) * 256,
                                    static_cast<cuuint64_t>(n_h) * 256};
     const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(group), 1, static_cast<cuuint32_t>(128 / group)};
-    if (enc(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(q), dims, strides, box, estr4,
+    if (enc(tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(q), dims, strides, box, estr4,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return false;
   }
   const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(n_kv), static_cast<cuuint64_t>(kv_rows)};
   const cuuint64_t strides[2] = {128 * 2, static_cast<cuuint64_t>(n_kv) * 256};
-  const cuuint32_t box[3] = {64, 1, 128};
   const void* src[2] = {k, v};
-  CUtensorMap* dst[2] = {&p.tm_k, &p.tm_v};
+  CUtensorMap* dst[2] = {tm_k, tm_v};
   for (int i = 0; i < 2; ++i) {
+    const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(i == 0 ? k_box_rows : 128)};
     if (enc(dst[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(src[i]), dims, strides, box, estr4,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -192,6 +195,13 @@ bool make_qkv_maps(tc::Params& p, const void* q, const void* k, const void* v, i
 }
 
 constexpr size_t kStatusBytes = 256;
+
+#ifndef CPK_PAIR_KERNEL
+#define CPK_PAIR_KERNEL 0
+#endif
+// bf16 partial attention on single SMs (default) or on SM pairs (cta_group::2,
+// built with -DCPK_PAIR_KERNEL=1: parity-tested, slower so far)
+constexpr bool kPairKernel = CPK_PAIR_KERNEL != 0;
 
 inline size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -333,11 +343,37 @@ static cp_status partial_impl(const void* q, const void* k, const void* v, cp_dt
   uint32_t* status = static_cast<uint32_t*>(workspace);
   const float log2e = 1.4426950408889634f;
 
-  if (dtype == CP_BF16) {
+  if (dtype == CP_BF16 && kPairKernel) {
+    static tc2::Params params;  // large: kept off the stack; copied at launch
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!make_qkv_maps(&params.tm_q, &params.tm_k, &params.tm_v, q, k, v, q_rows, kv_rows, n_h, n_kv, group, 64))
+      return CP_ERR_CUDA;
+    params.o_part = o_part;
+    params.lse_part = lse_part;
+    params.out_final = static_cast<__nv_bfloat16*>(out_final);
+    params.accumulate = accumulate != 0;
+    params.status = status;
+    params.n_h = n_h;
+    params.log2_group = ilog2_exact(group);
+    params.causal = causal != 0;
+    params.scale_log2 = softmax_scale * log2e;
+    if (cudaFuncSetAttribute(tc2::partial_bf16_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tc2::kSmemBytes) != cudaSuccess)
+      return CP_ERR_CUDA;
+    for (const WorkTable& wt : tables) {
+      if (wt.total_tiles == 0) continue;
+      std::memcpy(&params.wt, &wt, sizeof(WorkTable));
+      dim3 grid(2 * wt.total_tiles, n_kv);   // one cluster of two CTAs per 256-row tile
+      tc2::partial_bf16_pair_kernel<<<grid, tc2::kThreads, tc2::kSmemBytes, stream>>>(params);
+      if (last_cuda_status() != CP_OK) return CP_ERR_CUDA;
+    }
+  } else if (dtype == CP_BF16) {
     static tc::Params params;  // large: kept off the stack; copied at launch
     static std::mutex mu;
     std::lock_guard<std::mutex> lock(mu);
-    if (!make_qkv_maps(params, q, k, v, q_rows, kv_rows, n_h, n_kv, group)) return CP_ERR_CUDA;
+    if (!make_qkv_maps(&params.tm_q, &params.tm_k, &params.tm_v, q, k, v, q_rows, kv_rows, n_h, n_kv, group, 128))
+      return CP_ERR_CUDA;
     params.o_part = o_part;
     params.lse_part = lse_part;
     params.out_final = static_cast<__nv_bfloat16*>(out_final);
