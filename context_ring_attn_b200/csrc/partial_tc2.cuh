@@ -40,7 +40,7 @@
 //   warp 8      TMA producers of this CTA's halves: lane 0 Q and K, lane 1 V,
 //               signalling CTA 0's barriers;
 //   warp 9      TMEM owner (both CTAs) and, in CTA 0, the MMA issuer;
-//   warp 10     in CTA 1, the relay of P_FULL (below).
+//   warp 10     in CTA 1, the relay of P (below).
 // Cross-SM signals are few, since each costs: a commit multicast to both CTAs
 // holds the tensor pipe about 80 cycles, and a remote mbarrier arrive holds
 // the arriving thread about a thousand. So K and V use three stages, the
@@ -51,6 +51,11 @@
 // barrier; in CTA 1 one relay thread passes each completed step on to CTA 0
 // with a single remote arrive, off the softmax warps' path. Barriers that
 // collect both CTAs' loads (Q/K/V full) live in CTA 0.
+//
+// Launched only in a library built with CPK_PAIR_KERNEL=1. Measured on the
+// 128K causal prefill it is slower than the single-SM kernel (partial_tc.cuh):
+// the relayed arrive reaches CTA 0 thousands of cycles after the step, and the
+// issuer waits for it.
 #pragma once
 
 #include "common.cuh"
