@@ -146,3 +146,21 @@ def test_wait_selftest_rejects_bad_arguments(L):
     assert L.cp_wait_selftest(FAKE, 128, 1000, None) == B.CP_ERR_WORKSPACE
     assert L.cp_wait_selftest(FAKE, 256, 0, None) == B.CP_ERR_INVALID_ARG
     assert L.cp_wait_selftest(FAKE, 256, 2_000_000_000, None) == B.CP_ERR_INVALID_ARG
+
+
+def test_pair_kernel_build_compiles_and_exports(tmp_path):
+    """The opt-in SM-pair build (-DCPK_PAIR_KERNEL=1) compiles for sm_100a and
+    exports the same entry points."""
+    import subprocess
+    try:
+        nvcc = BUILD.nvcc_path()
+    except RuntimeError:
+        pytest.skip("nvcc not available")
+    out = str(tmp_path / "libcpattn_pair.so")
+    cmd = [nvcc, *BUILD.NVCC_FLAGS, "-DCPK_PAIR_KERNEL=1", "-I", BUILD.INCLUDE, "-I", BUILD.CSRC, "-o", out,
+           *[os.path.join(BUILD.CSRC, f) for f in BUILD.SOURCES]]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lib = ctypes.CDLL(out)
+    for n in header_functions():
+        assert hasattr(lib, n), n
