@@ -129,9 +129,14 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------ reference arm
-def oracle_sample(budget_s: float, seed_tokens: int = 0):
-    """Time the fp64 oracle on sampled query tokens of the 128K prefill (all 16
-    heads, each token against its causal prefix). Returns (flops, seconds, n_tokens)."""
+ORACLE_RUN = 256   # query rows per timed oracle call (the oracle's own row-group size)
+
+
+def oracle_sample(budget_s: float, seed: int = 0, min_runs: int = 1, max_runs: int | None = None):
+    """Time the fp64 oracle on runs of ORACLE_RUN consecutive query rows of the
+    128K prefill starting at seeded random positions (all 16 heads, each row
+    against its causal prefix), until budget_s of oracle time is spent and at
+    least min_runs runs are done. Returns (flops, seconds, n_rows)."""
     from context_ring_attn_b200 import synth
     from oracle import attention as OA
 
@@ -140,19 +145,64 @@ def oracle_sample(budget_s: float, seed_tokens: int = 0):
     k = synth.stored_values(synth.normal_rows(w["seed"], synth.TENSOR_K, t, (n_kv, d), w["std"]), "bf16")[0]
     v = synth.stored_values(synth.normal_rows(w["seed"], synth.TENSOR_V, t, (n_kv, d), w["std"]), "bf16")[0]
     k64, v64 = k.astype(np.float64), v.astype(np.float64)
-    rng = np.random.default_rng(12345 + seed_tokens)
-    flops, spent, n_tok = 0.0, 0.0, 0
+    rng = np.random.default_rng(12345 + seed)
+    flops, spent, n_rows, runs = 0.0, 0.0, 0, 0
     k_pos = np.arange(t)
-    while spent < budget_s or n_tok < 4:
-        tok = int(rng.integers(0, t))
-        qrow = synth.stored_values(synth.normal_rows(w["seed"], synth.TENSOR_Q, t, (n_h, d), w["std"], [tok]),
-                                   "bf16")[0]
+    while (spent < budget_s or runs < min_runs) and (max_runs is None or runs < max_runs):
+        r0 = int(rng.integers(0, t - ORACLE_RUN + 1))
+        rows = np.arange(r0, r0 + ORACLE_RUN)
+        q = synth.stored_values(synth.normal_rows(w["seed"], synth.TENSOR_Q, t, (n_h, d), w["std"], rows), "bf16")[0]
+        end = r0 + ORACLE_RUN
         t0 = time.perf_counter()
-        OA.attention(qrow, k64[:tok + 1], v64[:tok + 1], np.array([tok]), k_pos[:tok + 1])
+        OA.attention(q, k64[:end], v64[:end], rows, k_pos[:end])
         spent += time.perf_counter() - t0
-        flops += 4.0 * d * n_h * (tok + 1)
-        n_tok += 1
-    return flops, spent, n_tok
+        flops += 4.0 * d * n_h * float(np.sum(rows + 1))
+        n_rows += ORACLE_RUN
+        runs += 1
+    return flops, spent, n_rows
+
+
+SPEC = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}   # nominal dense bf16 and HBM3e of a B200
+
+
+def headline_config(t: int, n_h: int, n_kv: int, d: int, n_ranks: int, world: int) -> dict:
+    """The workload description both arms report (same keys, same values)."""
+    pairs = t * (t + 1) // 2
+    return {"workload": WORKLOAD if t == 131072 else f"{WORKLOAD} (T={t} profiling variant)",
+            "T": t, "N_H": n_h, "N_KV": n_kv, "D_H": d, "cp_ranks": n_ranks,
+            "plan": "load-balanced 16 chunks", "ring": "pass-KV", "merge": "final 8-way",
+            "flops_per_step": 4.0 * d * n_h * pairs, "causal_pairs_per_head": pairs,
+            "l2": "no flush: inputs larger than L2 (Q 537 MB, partials 8.6 GB per step)",
+            "parallelism": f"{world} independent replica(s)"}
+
+
+def peak_clock_mhz(peaks: dict):
+    """Median SM clock under which the measured peaks were taken, if the peaks
+    file records one (any numeric field whose name mentions a median SM clock)."""
+    def walk(obj, path=""):
+        if isinstance(obj, dict):
+            for k, v in obj.items():
+                yield from walk(v, f"{path}.{k}".lower())
+        elif isinstance(obj, (int, float)) and not isinstance(obj, bool):
+            yield path, float(obj)
+    cands = [(p, v) for p, v in walk(peaks) if ("mhz" in p or "clock" in p) and "median" in p and "max" not in p]
+    return cands[0][1] if cands else None
+
+
+def fractions(achieved: float, peak: float, spec: float, peaks: dict, clk) -> dict:
+    """achieved as a fraction of the measured peak, of the nominal spec peak,
+    and of the measured peak scaled to the clock the kernel ran at."""
+    out = {"frac_spec": achieved / spec, "spec_peak": spec}
+    pc = peak_clock_mhz(peaks)
+    run_mhz = (clk or {}).get("sm_mhz")
+    if pc and run_mhz:
+        out["frac_at_run_clock"] = achieved / (peak * run_mhz / pc)
+        out["peak_clock_mhz"] = pc
+        out["run_clock_mhz"] = run_mhz
+    else:
+        out["frac_at_run_clock"] = None
+        out["note"] = "the peaks file records no median SM clock: no clock-normalised fraction"
+    return out
 
 
 def blas_threads() -> int:
@@ -171,23 +221,23 @@ def run_reference(args, rank: int, world: int):
         return
     cores = blas_threads()
     per_step = max(2.0, min(8.0, 120.0 / max(1, args.steps)))
-    oracle_sample(0.5)  # warm caches and BLAS threads (not timed)
-    for _ in range(args.warmup):
-        oracle_sample(0.5)
+    oracle_sample(0.0, seed=1000, max_runs=1)  # warm caches and BLAS threads (not timed)
+    for i in range(args.warmup):
+        oracle_sample(0.0, seed=2000 + i, max_runs=1)
     flops = secs = 0.0
-    toks = 0
-    for _ in range(args.steps):
-        f, s, n = oracle_sample(per_step)
-        flops, secs, toks = flops + f, secs + s, toks + n
+    rows = 0
+    for i in range(args.steps):
+        f, s, n = oracle_sample(per_step, seed=i)
+        flops, secs, rows = flops + f, secs + s, rows + n
     value = flops / secs / 1e12
-    sample = (f"{toks} query tokens of the 128K causal prefill drawn at random positions, all 16 heads, "
-              f"fp64 numpy, each against its whole causal prefix; {args.steps} steps of ~{per_step:.0f} s")
+    sample = (f"{rows} query rows of the 128K causal prefill in runs of {ORACLE_RUN} consecutive rows at seeded "
+              f"random positions, all 16 heads, fp64 numpy, each row against its whole causal prefix; "
+              f"{args.steps} steps of >= {per_step:.0f} s")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "T": 131072, "N_H": 16, "N_KV": 1, "D_H": 128, "cp_ranks": 8,
-                   "plan": "load-balanced 16 chunks", "ring": "pass-KV"},
+        "config": headline_config(131072, 16, 1, 128, 8, world),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -227,10 +277,15 @@ def run_ours(args, rank: int, world: int):
     ev_part = []  # (start, end, flops) of each partial launch in the timed region
     ev_merge = []
 
+    nvtx = torch.cuda.nvtx
+
     def step(record: bool):
+        nvtx.range_push("plan")
         sched = ring.RingSchedule(segs, segs, n_ranks, B.CP_PASS_KV)   # host plan, every step
+        nvtx.range_pop()
         for s in range(n_ranks):
             blocks = sched.step_blocks(s, t)
+            nvtx.range_push(f"ring step {s}")
             if record:
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
@@ -239,6 +294,8 @@ def run_ours(args, rank: int, world: int):
             if record:
                 e1.record(stream)
                 ev_part.append((e0, e1, 4.0 * d * n_h * step_pairs[s]))
+            nvtx.range_pop()
+        nvtx.range_push("merge")
         if record:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
@@ -246,6 +303,7 @@ def run_ours(args, rank: int, world: int):
         if record:
             e1.record(stream)
             ev_merge.append((e0, e1))
+        nvtx.range_pop()
 
     def barrier():
         if world > 1:
@@ -313,6 +371,7 @@ def run_ours(args, rank: int, world: int):
     e2e = run_e2e(args, q, k, v, out, lse, o_parts, lse_parts, ws, segs, n_ranks, n_h, n_kv, world, dev,
                   step_flops, barrier) if not args.no_e2e else None
     decode = run_decode(args, dev) if not args.no_decode else None
+    context = run_library_context(args, dev) if not args.no_context else None
     secondary = {}
     if not args.no_secondary:
         for name in ("persistent_kv", "varlen_prefill"):
@@ -331,19 +390,16 @@ def run_ours(args, rank: int, world: int):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD if t == w["t"] else f"{WORKLOAD} (T={t} profiling variant)",
-                   "T": t, "N_H": n_h, "N_KV": n_kv, "D_H": d, "cp_ranks": n_ranks,
-                   "plan": "load-balanced 16 chunks", "ring": "pass-KV", "merge": "final 8-way",
-                   "flops_per_step": step_flops, "causal_pairs_per_head": pairs,
-                   "l2": "no flush: inputs larger than L2 (Q 537 MB, partials 8.6 GB per step)",
-                   "parallelism": f"{world} independent replica(s)"},
+        "config": headline_config(t, n_h, n_kv, d, n_ranks, world),
         "roofline": {"kernel": "partial_bf16_kernel", "bound": "tensor", "achieved": achieved, "peak": peak_t,
                      "unit": "TFLOP/s", "frac": achieved / peak_t, "traffic": traffic,
                      "peak_kind": f"bf16_tflops_sustained ({peak_kind})",
-                     "kernel_ms_per_step": part_ms / args.steps},
+                     "kernel_ms_per_step": part_ms / args.steps,
+                     **fractions(achieved, peak_t, SPEC["bf16_tflops"], peaks, clk)},
         "merge": {"ms_per_step": merge_ms / args.steps,
                   "gbs": merge_bytes / (merge_ms / args.steps * 1e-3) / 1e9,
-                  "frac_hbm": merge_bytes / (merge_ms / args.steps * 1e-3) / 1e9 / float(peaks["hbm_gbs"])},
+                  "frac_hbm": merge_bytes / (merge_ms / args.steps * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
+                  "frac_hbm_spec": merge_bytes / (merge_ms / args.steps * 1e-3) / 1e9 / SPEC["hbm_gbs"]},
         "fused_merge": None if fused_ms is None else {
             "value": world * step_flops / (fused_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": fused_ms,
             "note": "same step, LSE merge in the partial kernel's epilogue (cp_attn_partial_fused): "
@@ -354,14 +410,21 @@ def run_ours(args, rank: int, world: int):
     }
     if decode:
         line["decode"] = decode
+    if context:
+        line["library_context"] = context
     if secondary:
         line["workloads"] = secondary
     if not args.no_cpu_baseline:
-        f, s, n = oracle_sample(args.cpu_seconds)
+        f, s, n = oracle_sample(0.0, seed=0, min_runs=args.cpu_rows // ORACLE_RUN)
+        rate = f / s
         line["cpu_baseline"] = {
-            "value": f / s / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{n} query tokens of the 128K causal prefill at random positions, all 16 heads, fp64 numpy "
-                      f"against each token's causal prefix ({s:.1f} s)"}
+            "value": rate / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} query rows of the 128K causal prefill in runs of {ORACLE_RUN} consecutive rows at "
+                      f"seeded random positions, all 16 heads, fp64 numpy against each row's causal prefix "
+                      f"({s:.1f} s)",
+            "rows": n, "rows_per_s": n / s, "seconds": s,
+            "extrapolated_full_step_s": step_flops / rate,
+            "extrapolated_note": "extrapolated: one full 128K step's flops at the sampled rate"}
     print(json.dumps(line), flush=True)
 
 
@@ -562,12 +625,60 @@ def run_secondary(args, dev, name: str, merge_override: str | None = None):
            "flops_per_step": step_flops, "N_H": n_h, "N_KV": n_kv, "cp_ranks": n, **desc,
            "partial_tflops": step_flops / (part_ms * 1e-3) / 1e12,
            "partial_frac": step_flops / (part_ms * 1e-3) / 1e12 / peak_t,
+           "partial_frac_spec": step_flops / (part_ms * 1e-3) / 1e12 / SPEC["bf16_tflops"],
            "merge_gbs": None if no_merge else merge_bytes / (merge_ms * 1e-3) / 1e9,
            "merge_frac_hbm": None if no_merge else merge_bytes / (merge_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
            "peak_kind": f"bf16_tflops_sustained / hbm_gbs ({kind})"}
     del q, k, v, o_parts, lse_parts, out, lse
     torch.cuda.empty_cache()
     return res
+
+
+def run_library_context(args, dev):
+    """Context figure, not the product path: cuDNN's fused attention (torch's
+    scaled_dot_product_attention restricted to the cuDNN backend) on the same
+    causal 128K problem as one unsharded call, K/V expanded to the 16 query
+    heads, same bf16 inputs. Timed with CUDA events after warm-up."""
+    import torch
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+
+    from context_ring_attn_b200 import synth
+
+    w = synth.WORKLOADS[WORKLOAD]
+    t, n_h, d = w["t"], w["n_h"], w["d"]
+    if args.tokens:
+        t = args.tokens
+    try:
+        q = synth.device_rows(w["seed"], synth.TENSOR_Q, t, (n_h, d), w["std"], "bf16", dev)
+        k = synth.device_rows(w["seed"], synth.TENSOR_K, t, (1, d), w["std"], "bf16", dev)
+        v = synth.device_rows(w["seed"], synth.TENSOR_V, t, (1, d), w["std"], "bf16", dev)
+        qh = q.permute(1, 0, 2).unsqueeze(0).contiguous()
+        kh = k.permute(1, 0, 2).expand(n_h, t, d).unsqueeze(0).contiguous()
+        vh = v.permute(1, 0, 2).expand(n_h, t, d).unsqueeze(0).contiguous()
+        del q, k, v
+        stream = torch.cuda.current_stream()
+        with sdpa_kernel([SDPBackend.CUDNN_ATTENTION]):
+            for _ in range(2):
+                F.scaled_dot_product_attention(qh, kh, vh, is_causal=True)
+            torch.cuda.synchronize()
+            reps = 5
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                F.scaled_dot_product_attention(qh, kh, vh, is_causal=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        flops = 4.0 * d * n_h * t * (t + 1) / 2
+        del qh, kh, vh
+        torch.cuda.empty_cache()
+        return {"cudnn_sdpa": {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms": ms,
+                               "note": "context only: one unsharded causal call through cuDNN's fused attention "
+                                       "(torch SDPA, cuDNN backend), K/V expanded to 16 heads; not this library"}}
+    except Exception as exc:   # a missing backend is reported, not fatal
+        torch.cuda.empty_cache()
+        return {"cudnn_sdpa": {"unavailable": f"{type(exc).__name__}: {str(exc)[:200]}"}}
 
 
 def run_decode(args, dev):
@@ -645,6 +756,7 @@ def run_decode(args, dev):
     B.cp_check_status(ws_cp)
     return {"value": gbs, "unit": "GB/s", "ms": ms, "kv_bytes": kv_bytes, "batch": b, "n_splits": ns,
             "frac_hbm": gbs / float(peaks["hbm_gbs"]), "peak": float(peaks["hbm_gbs"]),
+            "frac_hbm_spec": gbs / SPEC["hbm_gbs"],
             "peak_kind": f"hbm_gbs ({kind})", "l2": "256 MB buffer written between iterations",
             "note": "balanced split kernel (8 ranges per SM) + per-head merge, median of iterations",
             "graph": {"ms": graph_ms, "value": kv_bytes / (graph_ms * 1e-3) / 1e9, "unit": "GB/s",
@@ -748,8 +860,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-rows", type=int, default=2048, help="query rows the CPU baseline times (runs of 256)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-context", action="store_true", help="skip the cuDNN context figure")
     ap.add_argument("--no-fused", action="store_true", help="skip timing the fused-merge variant of the step")
     ap.add_argument("--no-secondary", action="store_true", help="skip the persistent-KV and varlen workloads")
     ap.add_argument("--only-decode", action="store_true", help="time the split-KV decode workload alone")

@@ -44,7 +44,7 @@ EXPORTED = (
     "cp_classify_pair", "cp_block_pairs", "cp_ring_comm_volume", "cp_workspace_size",
     "cp_reset_status", "cp_check_status", "cp_attn_partial", "cp_attn_merge", "cp_decode",
     "cp_decode_static", "cp_decode_partial", "cp_select_ring_variant", "cp_attn_partial_fused",
-    "cp_wait_selftest",
+    "cp_wait_selftest", "cp_decode_static_status",
 )
 
 
@@ -85,7 +85,7 @@ def lib() -> ctypes.CDLL:
     sig = {
         "cp_status_string": (ctypes.c_char_p, [i32]),
         "cp_abi_version": (i32, []),
-        "cp_shard_plan": (i32, [P(cp_segment), i32, i32, i32, P(i64), P(i64), P(i64)]),
+        "cp_shard_plan": (i32, [P(cp_segment), i32, i32, i32, P(i64), P(i64), P(i64), P(i64)]),
         "cp_rank_ranges": (i32, [P(cp_segment), i32, i32, i32, i32, P(cp_range), P(i32)]),
         "cp_ring_schedule": (i32, [P(cp_segment), i32, P(cp_segment), i32, i32, i32, i32, P(cp_range), i32,
                                    P(i32), P(cp_block), P(i32)]),
@@ -103,6 +103,7 @@ def lib() -> ctypes.CDLL:
         "cp_attn_merge": (i32, [vp, vp, i32, i64, i64, i32, i32, vp, i32, vp, vp]),
         "cp_decode": (i32, [vp, vp, vp, i32, vp, i32, i64, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]),
         "cp_decode_static": (i32, [vp, vp, vp, i32, vp, i32, i64, i32, i32, i32, i32, f32, vp, vp, vp]),
+        "cp_decode_static_status": (i32, [vp]),
         "cp_select_ring_variant": (i32, [i64, i64, i32, i32, i32, i32, i32, ctypes.c_double, ctypes.c_double,
                                           vp, vp]),
         "cp_decode_partial": (i32, [vp, vp, vp, i32, vp, i32, i64, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]),
@@ -159,16 +160,26 @@ def cp_abi_version() -> int:
     return lib().cp_abi_version()
 
 
+def cp_shard_plan_sizes(segs, n_seg: int, n_ranks: int, mode: int):
+    """(len of chunk_bounds, len of rank_rows, len of token_index) for cp_shard_plan."""
+    sz = np.zeros(3, dtype=np.int64)
+    p64 = ctypes.POINTER(ctypes.c_int64)
+    _check("cp_shard_plan", lib().cp_shard_plan(segs, n_seg, n_ranks, mode, None, None, None,
+                                                sz.ctypes.data_as(p64)))
+    return tuple(int(x) for x in sz)
+
+
 def cp_shard_plan(segs, n_seg: int, n_ranks: int, mode: int):
-    """Returns (chunk_bounds [n_seg, 2N+1], rank_rows [N+1], token_index [sum len]) as int64 arrays."""
-    total = sum(segs[i].len for i in range(n_seg))
-    cb = np.zeros((max(1, n_seg), 2 * n_ranks + 1), dtype=np.int64)
-    rr = np.zeros(n_ranks + 1, dtype=np.int64)
-    ti = np.zeros(max(1, total), dtype=np.int64)
+    """Returns (chunk_bounds [n_seg, 2N+1], rank_rows [N+1], token_index [sum len]) as int64 arrays,
+    sized by the library's own sizes query."""
+    n_cb, n_rr, n_ti = cp_shard_plan_sizes(segs, n_seg, n_ranks, mode)
+    cb = np.zeros(max(1, n_cb), dtype=np.int64)
+    rr = np.zeros(n_rr, dtype=np.int64)
+    ti = np.zeros(max(1, n_ti), dtype=np.int64)
     p64 = ctypes.POINTER(ctypes.c_int64)
     _check("cp_shard_plan", lib().cp_shard_plan(segs, n_seg, n_ranks, mode, cb.ctypes.data_as(p64),
-                                                rr.ctypes.data_as(p64), ti.ctypes.data_as(p64)))
-    return cb[:n_seg], rr, ti[:total]
+                                                rr.ctypes.data_as(p64), ti.ctypes.data_as(p64), None))
+    return cb[:n_cb].reshape(n_seg, 2 * n_ranks + 1), rr, ti[:n_ti]
 
 
 def cp_rank_ranges(segs, n_seg: int, n_ranks: int, mode: int, rank: int):
@@ -297,9 +308,17 @@ def cp_decode_partial(q, k, v, kv_offsets, n_h: int, n_kv: int, n_splits: int, s
 def cp_decode_static(q, k, v, kv_offsets, n_h: int, n_kv: int, n_splits: int, softmax_scale: float, out, lse_out,
                      stream=None) -> None:
     """cp_decode without a workspace, for callers that cannot allocate device
-    memory while decoding: the split partials use the library's fixed 32 MiB
-    array on the current device. Calls must not overlap on the GPU."""
+    memory while decoding: the split partials and the status word use the
+    library's fixed 32 MiB array on the current device. Calls must not overlap
+    on the GPU; cp_decode_static_status reports the latest call's device-side
+    status."""
     code = lib().cp_decode_static(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(kv_offsets), int(q.shape[0]),
                                   int(k.shape[0]), n_h, n_kv, int(q.shape[-1]), n_splits, float(softmax_scale),
                                   _ptr(out), _ptr(lse_out), _stream(stream))
     _check("cp_decode_static", code)
+
+
+def cp_decode_static_status(stream=None) -> None:
+    """Synchronise the stream and raise CpError if the latest cp_decode_static
+    call on the current device recorded a device-side failure."""
+    _check("cp_decode_static_status", lib().cp_decode_static_status(_stream(stream)))

@@ -206,20 +206,136 @@ constexpr bool kPairKernel = CPK_PAIR_KERNEL != 0;
 inline size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Ranges of the flattened decode keys (one per warp of the persistent split
-// grid): 8 per SM of the current device, at most n_splits per (request, KV head).
-cp_status decode_ranges(int32_t n_splits, int32_t batch, int32_t n_kv, int32_t* n_warps) {
+// grid): 8 per SM of the current device, at most n_splits per flattened
+// (request, KV head, unit) triple.
+cp_status decode_ranges(int32_t n_splits, int32_t batch, int32_t triples_per_request, int32_t* n_warps) {
   int n_sm = 0, dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return CP_ERR_CUDA;
-  const int64_t want = (static_cast<int64_t>(n_splits) * batch * n_kv + 7) / 8;
+  const int64_t want = (static_cast<int64_t>(n_splits) * batch * triples_per_request + 7) / 8;
   *n_warps = static_cast<int32_t>(std::max<int64_t>(1, std::min<int64_t>(n_sm, want)) * 8);
   return CP_OK;
 }
 
-// Workspace bytes cp_decode uses with n_warps ranges (never above cp_workspace_size).
-size_t decode_ws_bytes(int32_t n_warps, int32_t batch, int32_t n_h, int32_t n_kv, int32_t d) {
-  const size_t part = (static_cast<size_t>(n_warps) + static_cast<size_t>(batch) * n_kv) * (n_h / n_kv);
-  return kStatusBytes + round256(part * d * 4) + round256(part * 4);
+// A decode call after its arguments have been checked: the unit split of the
+// query heads and the grid and workspace sizes it will use.
+struct DecodeShape {
+  int32_t group;    // G = n_h / n_kv
+  int32_t units;    // U: 16-head units per KV head (1 for G <= 16)
+  int32_t rows;     // R: partial rows per slot, min(G, 16)
+  int32_t n_warps;  // W: ranges of the flattened keys
+  size_t part_rows; // (W + batch * n_kv * U) * R
+  size_t bytes;     // workspace bytes the call uses (never above cp_workspace_size)
+};
+
+// Every argument check of cp_decode / cp_decode_partial / cp_decode_static,
+// with nothing launched, nothing written and no CUDA call; fills in the unit
+// split of the query heads.
+cp_status decode_validate(const void* q, const void* k, const void* v, cp_dtype dtype, const int64_t* kv_offsets,
+                          int32_t batch, int64_t kv_rows, int32_t n_h, int32_t n_kv, int32_t d, int32_t n_splits,
+                          float softmax_scale, const void* out, bool out_f32, DecodeShape* s) {
+  if (!q || !k || !v || !kv_offsets || !out) return CP_ERR_INVALID_ARG;
+  if (batch < 0 || kv_rows < 0 || n_h < 1 || n_kv < 1 || d < 1 || n_h % n_kv) return CP_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.0f) || !(softmax_scale < INFINITY)) return CP_ERR_INVALID_ARG;
+  if (n_splits < 1 || n_splits > dec::kMaxSplits) return CP_ERR_UNSUPPORTED;
+  const int group = n_h / n_kv;
+  if (dtype != CP_BF16 || (d != 64 && d != 128)) return CP_ERR_UNSUPPORTED;
+  if (group > 128 || (group > dec::kUnitRows && group % dec::kUnitRows != 0)) return CP_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(batch) * n_h > 0x7fffffffLL) return CP_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, out_f32 ? 16 : 8) || !aligned(kv_offsets, 8))
+    return CP_ERR_INVALID_ARG;
+  s->group = group;
+  s->units = group > dec::kUnitRows ? group / dec::kUnitRows : 1;
+  s->rows = group > dec::kUnitRows ? dec::kUnitRows : group;
+  s->n_warps = 0;
+  s->part_rows = 0;
+  s->bytes = 0;
+  return CP_OK;
+}
+
+// Partial rows and workspace bytes of a decode with n_warps ranges.
+void decode_sizes(DecodeShape* s, int32_t n_warps, int32_t batch, int32_t n_kv, int32_t d) {
+  s->n_warps = n_warps;
+  s->part_rows = (static_cast<size_t>(n_warps) + static_cast<size_t>(batch) * n_kv * s->units) * s->rows;
+  s->bytes = kStatusBytes + round256(s->part_rows * d * 4) + round256(s->part_rows * 4);
+}
+
+// Grid of the current device (the one CUDA query of a decode call before its
+// launches) and the sizes that follow from it.
+cp_status decode_grid(DecodeShape* s, int32_t n_splits, int32_t batch, int64_t kv_rows, int32_t n_kv, int32_t d) {
+  int32_t n_warps = 0;
+  if (decode_ranges(n_splits, batch, n_kv * s->units, &n_warps) != CP_OK) return CP_ERR_CUDA;
+  // the range arithmetic is exact while (flattened keys) x W stays below 2^53
+  const double kt_max = static_cast<double>(kv_rows) * n_kv * s->units;
+  if (kt_max * (static_cast<double>(n_warps) + 1.0) >= 9007199254740992.0) return CP_ERR_UNSUPPORTED;
+  decode_sizes(s, n_warps, batch, n_kv, d);
+  return CP_OK;
+}
+
+// Launch the split kernel and, as its programmatic dependent, the merge. The
+// status word is at `ws`, the partials follow it.
+template <int D>
+cp_status decode_launch_d(const DecodeShape& s, const void* q, const void* k, const void* v,
+                                 const int64_t* kv_offsets, int32_t batch, int64_t kv_rows, int32_t n_h, int32_t n_kv,
+                                 float softmax_scale, void* out, bool out_f32, float* lse_out, void* ws,
+                                 cudaStream_t stream) {
+  float* o_ws = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kStatusBytes);
+  float* l_ws = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kStatusBytes + round256(s.part_rows * D * 4));
+  dec::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.offsets = kv_offsets;
+  p.kv_rows = kv_rows;
+  p.o_part = o_ws;
+  p.lse_part = l_ws;
+  p.status = static_cast<uint32_t*>(ws);
+  p.batch = batch;
+  p.n_h = n_h;
+  p.n_kv = n_kv;
+  p.group = s.group;
+  p.units = s.units;
+  p.rows = s.rows;
+  p.n_warps = s.n_warps;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  if (cudaFuncSetAttribute(dec::decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           dec::kSmemBytes) != cudaSuccess)
+    return CP_ERR_CUDA;
+  // persistent: up to one CTA per SM, each warp streaming one range of the flattened keys
+  dec::decode_split_kernel<D><<<static_cast<unsigned>(s.n_warps / dec::kWarps), dec::kThreads, dec::kSmemBytes, stream>>>(p);
+  if (last_cuda_status() != CP_OK) return CP_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(static_cast<int64_t>(batch) * n_h));
+  cfg.blockDim = dim3(dec::kMergeThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
+  if (out_f32)
+    e = cudaLaunchKernelEx(&cfg, dec::decode_merge_kernel<float, D>, p, static_cast<float*>(out), lse_out);
+  else
+    e = cudaLaunchKernelEx(&cfg, dec::decode_merge_kernel<__nv_bfloat16, D>, p, static_cast<__nv_bfloat16*>(out),
+                           lse_out);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return CP_ERR_CUDA;
+  }
+  return last_cuda_status();
+}
+
+cp_status decode_launch(const DecodeShape& s, const void* q, const void* k, const void* v,
+                               const int64_t* kv_offsets, int32_t batch, int64_t kv_rows, int32_t n_h, int32_t n_kv,
+                               int32_t d, float softmax_scale, void* out, bool out_f32, float* lse_out, void* ws,
+                               cudaStream_t stream) {
+  if (d == 64)
+    return decode_launch_d<64>(s, q, k, v, kv_offsets, batch, kv_rows, n_h, n_kv, softmax_scale, out, out_f32,
+                               lse_out, ws, stream);
+  return decode_launch_d<128>(s, q, k, v, kv_offsets, batch, kv_rows, n_h, n_kv, softmax_scale, out, out_f32,
+                              lse_out, ws, stream);
 }
 
 }  // namespace
@@ -484,56 +600,21 @@ cp_status cp_attn_merge(const float* o_parts, const float* lse_parts, int32_t n_
 }
 
 static cp_status decode_impl(const void* q, const void* k, const void* v, cp_dtype dtype, const int64_t* kv_offsets,
-                    int32_t batch, int64_t kv_rows, int32_t n_h, int32_t n_kv, int32_t d, int32_t n_splits,
-                    float softmax_scale, void* out, bool out_f32, float* lse_out, void* workspace, size_t ws_bytes,
-                    void* cuda_stream) {
-  if (!q || !k || !v || !kv_offsets || !out) return CP_ERR_INVALID_ARG;
-  if (batch < 0 || kv_rows < 0 || n_h < 1 || n_kv < 1 || d < 1 || n_h % n_kv) return CP_ERR_INVALID_ARG;
-  if (!(softmax_scale > 0.0f) || !(softmax_scale < INFINITY)) return CP_ERR_INVALID_ARG;
-  if (n_splits < 1 || n_splits > dec::kMaxSplits) return CP_ERR_UNSUPPORTED;
-  const int group = n_h / n_kv;
-  if (dtype != CP_BF16 || d != 128 || group > 16 || (16 % group) != 0) return CP_ERR_UNSUPPORTED;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, out_f32 ? 16 : 8) || !aligned(kv_offsets, 8))
-    return CP_ERR_INVALID_ARG;
-  if (!workspace || !aligned(workspace, 256) || ws_bytes < decode_ws_bytes(dec::kWarps, batch, n_h, n_kv, d))
-    return CP_ERR_WORKSPACE;   // below what even the smallest grid needs
+                             int32_t batch, int64_t kv_rows, int32_t n_h, int32_t n_kv, int32_t d, int32_t n_splits,
+                             float softmax_scale, void* out, bool out_f32, float* lse_out, void* workspace,
+                             size_t ws_bytes, void* cuda_stream) {
+  DecodeShape s;
+  cp_status st = decode_validate(q, k, v, dtype, kv_offsets, batch, kv_rows, n_h, n_kv, d, n_splits, softmax_scale,
+                                 out, out_f32, &s);
+  if (st != CP_OK) return st;
+  decode_sizes(&s, dec::kWarps, batch, n_kv, d);   // below what even the smallest grid needs
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < s.bytes) return CP_ERR_WORKSPACE;
+  st = decode_grid(&s, n_splits, batch, kv_rows, n_kv, d);
+  if (st != CP_OK) return st;
+  if (ws_bytes < s.bytes) return CP_ERR_WORKSPACE;
   if (batch == 0) return CP_OK;
-  int32_t n_warps = 0;
-  if (decode_ranges(n_splits, batch, n_kv, &n_warps) != CP_OK) return CP_ERR_CUDA;
-  if (ws_bytes < decode_ws_bytes(n_warps, batch, n_h, n_kv, d)) return CP_ERR_WORKSPACE;
-  const size_t part = (static_cast<size_t>(n_warps) + static_cast<size_t>(batch) * n_kv) * group;
-  float* o_ws = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
-  float* l_ws = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes + round256(part * d * 4));
-  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-  dec::Params p;
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.k = static_cast<const __nv_bfloat16*>(k);
-  p.v = static_cast<const __nv_bfloat16*>(v);
-  p.offsets = kv_offsets;
-  p.kv_rows = kv_rows;
-  p.o_part = o_ws;
-  p.lse_part = l_ws;
-  p.status = static_cast<uint32_t*>(workspace);
-  p.batch = batch;
-  p.n_h = n_h;
-  p.n_kv = n_kv;
-  p.group = group;
-  p.n_warps = n_warps;
-  p.scale_log2 = softmax_scale * 1.4426950408889634f;
-  if (cudaFuncSetAttribute(dec::decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           dec::kSmemBytes) != cudaSuccess)
-    return CP_ERR_CUDA;
-  // persistent: up to one CTA per SM, each warp streaming one range of the flattened keys
-  dec::decode_split_kernel<<<static_cast<unsigned>(n_warps / dec::kWarps), dec::kThreads, dec::kSmemBytes, stream>>>(p);
-  if (last_cuda_status() != CP_OK) return CP_ERR_CUDA;
-  const int64_t n_rowheads = static_cast<int64_t>(batch) * n_h;
-  if (out_f32)
-    dec::decode_merge_kernel<float><<<static_cast<unsigned>(n_rowheads), dec::kMergeThreads, 0, stream>>>(
-        p, static_cast<float*>(out), lse_out);
-  else
-    dec::decode_merge_kernel<__nv_bfloat16><<<static_cast<unsigned>(n_rowheads), dec::kMergeThreads, 0, stream>>>(
-        p, static_cast<__nv_bfloat16*>(out), lse_out);
-  return last_cuda_status();
+  return decode_launch(s, q, k, v, kv_offsets, batch, kv_rows, n_h, n_kv, d, softmax_scale, out, out_f32, lse_out,
+                       workspace, static_cast<cudaStream_t>(cuda_stream));
 }
 
 cp_status cp_decode(const void* q, const void* k, const void* v, cp_dtype dtype, const int64_t* kv_offsets,
@@ -594,17 +675,30 @@ extern "C" cp_status cp_decode_static(const void* q, const void* k, const void* 
                                       const int64_t* kv_offsets, int32_t batch, int64_t kv_rows, int32_t n_h,
                                       int32_t n_kv, int32_t d, int32_t n_splits, float softmax_scale, void* out,
                                       float* lse_out, void* cuda_stream) {
-  if (batch < 0 || n_h < 1 || n_kv < 1 || d < 1 || n_splits < 1 || n_h % n_kv) return CP_ERR_INVALID_ARG;
-  if (n_splits > dec::kMaxSplits) return CP_ERR_UNSUPPORTED;
-  int32_t n_warps = 0;
-  if (decode_ranges(n_splits, batch, n_kv, &n_warps) != CP_OK) return CP_ERR_CUDA;
-  if (decode_ws_bytes(n_warps, batch, n_h, n_kv, d) > kStaticScratchBytes) return CP_ERR_WORKSPACE;
+  // every argument is checked before anything is enqueued
+  DecodeShape s;
+  cp_status st = decode_validate(q, k, v, dtype, kv_offsets, batch, kv_rows, n_h, n_kv, d, n_splits, softmax_scale,
+                                 out, false, &s);
+  if (st != CP_OK) return st;
+  st = decode_grid(&s, n_splits, batch, kv_rows, n_kv, d);
+  if (st != CP_OK) return st;
+  if (s.bytes > kStaticScratchBytes) return CP_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  st = scratch_for_current_device(&scratch);
+  if (st != CP_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  // The status word starts at zero for every call (so that
+  // cp_decode_static_status reports this call); the split partials are fully
+  // rewritten before the merge reads them.
+  if (cudaMemsetAsync(scratch, 0, sizeof(uint32_t), stream) != cudaSuccess) return CP_ERR_CUDA;
+  if (batch == 0) return CP_OK;
+  return decode_launch(s, q, k, v, kv_offsets, batch, kv_rows, n_h, n_kv, d, softmax_scale, out, false, lse_out,
+                       scratch, stream);
+}
+
+extern "C" cp_status cp_decode_static_status(void* cuda_stream) {
   void* scratch = nullptr;
   const cp_status st = scratch_for_current_device(&scratch);
   if (st != CP_OK) return st;
-  // The status word must start at zero; the split partials are fully rewritten.
-  if (cudaMemsetAsync(scratch, 0, sizeof(uint32_t), static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
-    return CP_ERR_CUDA;
-  return cp_decode(q, k, v, dtype, kv_offsets, batch, kv_rows, n_h, n_kv, d, n_splits, softmax_scale, out, lse_out,
-                   scratch, kStaticScratchBytes, cuda_stream);
+  return cp_check_status(scratch, cuda_stream);
 }

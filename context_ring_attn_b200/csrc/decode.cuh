@@ -6,21 +6,28 @@
 //
 // The work is HBM-bound (every K/V byte is read once; 16 flop per byte with
 // 16 query heads per KV head), so the design goal is streaming K/V at full
-// bandwidth with the least fixed cost and no tail. The splits are cut over
-// the whole batch: the keys of all (request, KV head) pairs, in order, form
-// one flattened sequence of Kt = n_kv * (offsets[B] - offsets[0]) keys, and
-// warp w of the persistent grid of W warps owns the range
-// [w*Kt/W, (w+1)*Kt/W). Every warp thus streams the same number of keys
-// (within one key), whatever the mix of request lengths, and writes one
-// partial per (request, KV head) its range overlaps: about W + B*n_kv
-// partials in all. Warp w's partial for pair bg lands in slot w + bg, which is
-// unique because both the ranges and the pairs are in flattened order.
+// bandwidth with the least fixed cost and no tail.
 //
-// Each warp works alone: a private 3-stage ring of 16-key steps of K and V in
-// shared memory, filled by 16-byte cp.async copies (rows of 256 bytes, fully
-// coalesced) that run ahead across pair boundaries. All G <= 16 query heads
-// of the KV head share every K/V load: they are the 16 rows of m16n8k16 bf16
-// MMAs (S = q K^T, then O += P V with P kept in registers).
+// Units. The query heads of one KV head are taken 16 at a time: a group of
+// G <= 16 heads is one unit (rows past G are zero), a group of G = 16u heads
+// is u units that each stream the KV head's keys (GQA section 8.2 of the GQA
+// page: heads h of one group share the KV head floor(h / G)).
+//
+// The splits are cut over the whole batch: the keys of all (request, KV head,
+// unit) triples, in order, form one flattened sequence of
+// Kt = n_kv * U * (offsets[B] - offsets[0]) keys, and warp w of the persistent
+// grid of W warps owns the range [w*Kt/W, (w+1)*Kt/W). Every warp thus streams
+// the same number of keys (within one key), whatever the mix of request
+// lengths, and writes one partial per triple its range overlaps: about
+// W + B*n_kv*U partials in all. Warp w's partial for triple bg lands in slot
+// w + bg, which is unique because both the ranges and the triples are in
+// flattened order.
+//
+// Each warp works alone: a private ring of 16-key steps of K and V in shared
+// memory, filled by 16-byte cp.async copies (whole key rows, fully coalesced)
+// that run ahead across triple boundaries. The 16 query heads of a unit share
+// every K/V load: they are the 16 rows of m16n8k16 bf16 MMAs (S = q K^T, then
+// O += P V with P kept in registers).
 #pragma once
 
 #include "common.cuh"
@@ -31,12 +38,19 @@ namespace dec {
 constexpr int kWarps = 8;                 // warps per CTA, one CTA per SM
 constexpr int kThreads = kWarps * 32;
 constexpr int kStepKeys = 16;             // keys per pipeline step of a warp
-constexpr int kStages = 3;                // steps in flight per warp
-constexpr int kRowBytes = 256;            // 128 bf16
-constexpr int kStepBytes = 2 * kStepKeys * kRowBytes;   // K + V of one step: 8 KB
-constexpr int kWarpBytes = kStages * kStepBytes;        // 24 KB per warp
-constexpr int kSmemBytes = kWarps * kWarpBytes;         // 192 KB
+constexpr int kWarpBytes = 24 * 1024;     // shared ring per warp (K + V steps in flight)
+constexpr int kSmemBytes = kWarps * kWarpBytes;   // 192 KB
 constexpr int kMaxSplits = 1024;
+constexpr int kUnitRows = 16;             // query heads per unit (MMA rows)
+
+template <int D>
+struct Cfg {
+  static constexpr int kRowBytes = D * 2;                        // one key row of K (or V), bf16
+  static constexpr int kChunks = D / 8;                          // 16-byte chunks per row
+  static constexpr int kStepBytes = 2 * kStepKeys * kRowBytes;   // K + V of one step: 4 or 8 KB
+  static constexpr int kStages = kWarpBytes / kStepBytes;        // 6 or 3 steps in flight
+  static_assert(kStages >= 3, "ring too shallow");
+};
 
 struct Params {
   const __nv_bfloat16* q;
@@ -44,13 +58,15 @@ struct Params {
   const __nv_bfloat16* v;
   const int64_t* offsets;
   int64_t kv_rows;
-  float* o_part;   // [slot][G][128], slot = warp + pair
-  float* lse_part; // [slot][G]
+  float* o_part;   // [slot][R][D], slot = warp + triple
+  float* lse_part; // [slot][R]
   uint32_t* status;
   int32_t batch;
   int32_t n_h;
   int32_t n_kv;
-  int32_t group;
+  int32_t group;   // G = n_h / n_kv
+  int32_t units;   // U: units per KV head (1 for G <= 16, G / 16 above)
+  int32_t rows;    // R: partial rows per slot, min(G, 16)
   int32_t n_warps; // W: warps of the split grid = ranges of the flattened keys
   float scale_log2;
 };
@@ -84,8 +100,12 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// byte offset of 16-byte chunk c of key row r inside a K or V step
-__device__ __forceinline__ uint32_t swz(int r, int c) { return r * kRowBytes + ((c ^ (r & 7)) << 4); }
+// byte offset of 16-byte chunk c of key row r inside a K or V step (rows of
+// `row_bytes`, chunks XOR-swizzled by the row so ldmatrix is conflict-free)
+template <int D>
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+  return r * Cfg<D>::kRowBytes + ((c ^ (r & 7)) << 4);
+}
 
 // floor(x / y) for 0 <= x < 2^53, 0 < y < 2^53, exactly: the double quotient
 // is correctly rounded, so its truncation is the true quotient or one above it
@@ -105,18 +125,19 @@ __device__ __forceinline__ int64_t range_of(int64_t x, int64_t kt, int64_t n) {
   return w < n - 1 ? w : n - 1;
 }
 
-// Part of one warp's range inside one (request, KV head) pair.
+// Part of one warp's range inside one (request, KV head, unit) triple.
 struct Piece {
   int64_t row0;  // first K/V row
   int n_keys;
-  int b, g, bg;
+  int b, g, u, bg;
 };
 
-// Walks the pairs that overlap [a, e) in flattened order. Every pair it looks
-// at is checked (rows inside [0, kv_rows)), so the walk stays in bounds even
-// for offsets that break the non-decreasing contract; the merge reports those.
+// Walks the triples that overlap [a, e) in flattened order. Every triple it
+// looks at is checked (rows inside [0, kv_rows)), so the walk stays in bounds
+// even for offsets that break the non-decreasing contract; the merge reports
+// those.
 struct Walker {
-  int bg;        // next pair to look at
+  int bg;        // next triple to look at
   int64_t a, e;  // the range
   int64_t o0;    // offsets[0]
 
@@ -124,32 +145,34 @@ struct Walker {
     a = a_;
     e = e_;
     o0 = o0_;
+    const int64_t per_tok = static_cast<int64_t>(p.n_kv) * p.units;   // flattened keys per token row
     int lo = 0, hi = p.batch - 1;   // last request whose first flattened key is <= a
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if ((p.offsets[mid] - o0) * p.n_kv <= a) lo = mid;
+      if ((p.offsets[mid] - o0) * per_tok <= a) lo = mid;
       else hi = mid - 1;
     }
     const int64_t base = p.offsets[lo], len = p.offsets[lo + 1] - base;
-    int64_t g = 0;
+    int64_t gu = 0;
     if (len > 0) {
-      g = (a - (base - o0) * p.n_kv) / len;
-      g = g < 0 ? 0 : (g >= p.n_kv ? p.n_kv - 1 : g);
+      gu = (a - (base - o0) * per_tok) / len;
+      gu = gu < 0 ? 0 : (gu >= per_tok ? per_tok - 1 : gu);
     }
-    bg = lo * p.n_kv + static_cast<int>(g);
+    bg = lo * static_cast<int>(per_tok) + static_cast<int>(gu);
   }
 
   // next non-empty piece; false once the range is done
   __device__ __forceinline__ bool next(const Params& p, Piece& t) {
-    const int n_bg = p.batch * p.n_kv;
+    const int per_tok = p.n_kv * p.units;
+    const int n_bg = p.batch * per_tok;
     while (bg < n_bg) {
       const int cur = bg++;
-      const int b = cur / p.n_kv;
-      const int g = cur - b * p.n_kv;
+      const int b = cur / per_tok;
+      const int gu = cur - b * per_tok;
       const int64_t base = p.offsets[b], end = p.offsets[b + 1];
       if (!(base >= o0 && end >= base && end <= p.kv_rows)) continue;
       const int64_t len = end - base;
-      const int64_t vs = (base - o0) * p.n_kv + g * len;
+      const int64_t vs = (base - o0) * per_tok + gu * len;
       if (vs >= e) {
         bg = n_bg;
         return false;
@@ -160,7 +183,8 @@ struct Walker {
         t.row0 = base + (lo - vs);
         t.n_keys = static_cast<int>(hi - lo);
         t.b = b;
-        t.g = g;
+        t.g = gu / p.units;
+        t.u = gu - t.g * p.units;
         t.bg = cur;
         return true;
       }
@@ -169,21 +193,32 @@ struct Walker {
   }
 };
 
+// Let the merge launch (a programmatic dependent of this grid) start its
+// blocks early: they wait in griddepcontrol.wait until this grid has finished
+// and its writes are visible, so the launch gap is hidden.
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_constant__ Params p) {
+  using C = Cfg<D>;
+  constexpr int KS = D / 16;   // k-steps of the S product
+  constexpr int NT = D / 8;    // 8-wide column tiles of O
   extern __shared__ __align__(128) uint8_t smem[];
+  allow_dependents();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int gw = blockIdx.x * kWarps + warp;
   const uint32_t ring = smem_u32(smem) + warp * kWarpBytes;
-  const int row_stride = p.n_kv * 128;   // elements between consecutive keys
+  const int row_stride = p.n_kv * D;   // elements between consecutive keys
   const float sl2 = p.scale_log2;
-  const int gr = lane >> 2;  // fragment row (query head in the group)
+  const int gr = lane >> 2;  // fragment row (query head in the unit)
   const int tq = lane & 3;   // fragment column pair
 
   const int64_t o0 = p.offsets[0];
   const int64_t oB = p.offsets[p.batch];
   if (!(o0 >= 0 && oB >= o0 && oB <= p.kv_rows)) return;   // reported by the merge
-  const int64_t kt = (oB - o0) * p.n_kv;
+  const int64_t kt = (oB - o0) * p.n_kv * p.units;
   if (kt == 0) return;
   const int64_t a = range_start(gw, kt, p.n_warps);
   const int64_t e = range_start(gw + 1, kt, p.n_warps);
@@ -197,21 +232,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
   int l_slot = 0;
   auto issue_step = [&]() {   // copies of one step, or nothing once the range is done
     if (l_more) {
-      const uint32_t sk = ring + l_slot * kStepBytes;
-      const uint32_t sv = sk + kStepKeys * kRowBytes;
+      const uint32_t sk = ring + l_slot * C::kStepBytes;
+      const uint32_t sv = sk + kStepKeys * C::kRowBytes;
 #pragma unroll
-      for (int i = 0; i < (kStepKeys * 16) / 32; ++i) {
-        const int c = lane + i * 32;   // 16-byte chunk of the 16 x 256-byte step
-        const int r = c >> 4;
-        const int cc = c & 15;
+      for (int i = 0; i < (kStepKeys * C::kChunks) / 32; ++i) {
+        const int c = lane + i * 32;   // 16-byte chunk of the step's rows
+        const int r = c / C::kChunks;
+        const int cc = c % C::kChunks;
         const int kr = l_step * kStepKeys + r;
         const bool in = kr < lp.n_keys;
         const int64_t row = in ? lp.row0 + kr : 0;
-        const size_t off = static_cast<size_t>(row) * row_stride + lp.g * 128 + cc * 8;
-        cp_async16(sk + swz(r, cc), p.k + off, in ? 16u : 0u);
-        cp_async16(sv + swz(r, cc), p.v + off, in ? 16u : 0u);
+        const size_t off = static_cast<size_t>(row) * row_stride + lp.g * D + cc * 8;
+        cp_async16(sk + swz<D>(r, cc), p.k + off, in ? 16u : 0u);
+        cp_async16(sv + swz<D>(r, cc), p.v + off, in ? 16u : 0u);
       }
-      l_slot = (l_slot + 1) % kStages;
+      l_slot = (l_slot + 1) % C::kStages;
       if (++l_step * kStepKeys >= lp.n_keys) {
         l_step = 0;
         l_more = lw.next(p, lp);
@@ -220,42 +255,43 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
     cp_async_commit();
   };
 #pragma unroll
-  for (int s = 0; s < kStages - 1; ++s) issue_step();
+  for (int s = 0; s < C::kStages - 1; ++s) issue_step();
 
   Walker cw;
   cw.init(p, a, e, o0);
   Piece t;
   int c_slot = 0;
   while (cw.next(p, t)) {
-    const size_t prow = static_cast<size_t>(gw + t.bg) * p.group;   // first partial row of this piece
-    // Q fragments: rows = query heads of the group (rows >= G are zero), 8 k-steps of 16 dims
-    uint32_t qa[8][4];
+    const size_t prow = static_cast<size_t>(gw + t.bg) * p.rows;   // first partial row of this piece
+    // Q fragments: rows = the unit's query heads (rows past the group are zero), D/16 k-steps
+    const int h_first = t.u * kUnitRows;   // first head of the unit within the group
+    const bool r0 = h_first + gr < p.group, r1 = h_first + gr + 8 < p.group;
+    uint32_t qa[KS][4];
     {
-      const __nv_bfloat16* qb = p.q + (static_cast<size_t>(t.b) * p.n_h + t.g * p.group) * 128;
-      const bool r0 = gr < p.group, r1 = gr + 8 < p.group;
+      const __nv_bfloat16* qb = p.q + (static_cast<size_t>(t.b) * p.n_h + t.g * p.group + h_first) * D;
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
+      for (int ks = 0; ks < KS; ++ks) {
         const int c0 = ks * 16 + tq * 2;
-        qa[ks][0] = r0 ? *reinterpret_cast<const uint32_t*>(qb + gr * 128 + c0) : 0u;
-        qa[ks][1] = r1 ? *reinterpret_cast<const uint32_t*>(qb + (gr + 8) * 128 + c0) : 0u;
-        qa[ks][2] = r0 ? *reinterpret_cast<const uint32_t*>(qb + gr * 128 + c0 + 8) : 0u;
-        qa[ks][3] = r1 ? *reinterpret_cast<const uint32_t*>(qb + (gr + 8) * 128 + c0 + 8) : 0u;
+        qa[ks][0] = r0 ? *reinterpret_cast<const uint32_t*>(qb + gr * D + c0) : 0u;
+        qa[ks][1] = r1 ? *reinterpret_cast<const uint32_t*>(qb + (gr + 8) * D + c0) : 0u;
+        qa[ks][2] = r0 ? *reinterpret_cast<const uint32_t*>(qb + gr * D + c0 + 8) : 0u;
+        qa[ks][3] = r1 ? *reinterpret_cast<const uint32_t*>(qb + (gr + 8) * D + c0 + 8) : 0u;
       }
     }
-    float o[16][4];
+    float o[NT][4];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.0f;
+    for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.0f;
     float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 units) of rows gr, gr+8
     float l0 = 0.0f, l1 = 0.0f;            // thread-partial running sums
     const int n_steps = (t.n_keys + kStepKeys - 1) / kStepKeys;
 
     for (int st = 0; st < n_steps; ++st) {
-      cp_async_wait<kStages - 2>();
+      cp_async_wait<C::kStages - 2>();
       __syncwarp();
       issue_step();
-      const uint32_t sk = ring + c_slot * kStepBytes;
-      const uint32_t sv = sk + kStepKeys * kRowBytes;
-      c_slot = (c_slot + 1) % kStages;
+      const uint32_t sk = ring + c_slot * C::kStepBytes;
+      const uint32_t sv = sk + kStepKeys * C::kRowBytes;
+      c_slot = (c_slot + 1) % C::kStages;
 
       // S = Q K^T for 16 keys: two n-tiles of 8 keys
       float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -263,9 +299,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
         const int mi = lane >> 3, rr = lane & 7;
         const int key = (mi >> 1) * 8 + rr;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
+        for (int ks = 0; ks < KS; ++ks) {
           uint32_t b0, b1, b2, b3;
-          ldsm_x4(sk + swz(key, ks * 2 + (mi & 1)), b0, b1, b2, b3);
+          ldsm_x4(sk + swz<D>(key, ks * 2 + (mi & 1)), b0, b1, b2, b3);
           mma16816(s[0], qa[ks], b0, b1);
           mma16816(s[1], qa[ks], b2, b3);
         }
@@ -303,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
       l0 = l0 * a0 + pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1];
       l1 = l1 * a1 + pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < NT; ++j) {
         o[j][0] *= a0;
         o[j][1] *= a0;
         o[j][2] *= a1;
@@ -314,38 +350,38 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
       pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
       pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
       pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
-      // O += P V: 16 d-tiles of 8, two per transposed ldmatrix.x4
+      // O += P V: D/8 column tiles of 8, two per transposed ldmatrix.x4
       {
         const int mi = lane >> 3, rr = lane & 7;
         const int key = (mi & 1) * 8 + rr;
 #pragma unroll
-        for (int j = 0; j < 16; j += 2) {
+        for (int j = 0; j < NT; j += 2) {
           uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(sv + swz(key, j + (mi >> 1)), b0, b1, b2, b3);
+          ldsm_x4_t(sv + swz<D>(key, j + (mi >> 1)), b0, b1, b2, b3);
           mma16816(o[j], pa, b0, b1);
           mma16816(o[j + 1], pa, b2, b3);
         }
       }
       __syncwarp();   // this slot is refilled only after every lane has read it
     }
-    // partial of this piece: normalise and write rows < G
+    // partial of this piece: normalise and write the unit's rows
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
     const float inv0 = (l0 > 0.0f) ? 1.0f / l0 : 0.0f;
     const float inv1 = (l1 > 0.0f) ? 1.0f / l1 : 0.0f;
-    if (gr < p.group) {
-      float* dst = p.o_part + (prow + gr) * 128;
+    if (r0) {
+      float* dst = p.o_part + (prow + gr) * D;
 #pragma unroll
-      for (int j = 0; j < 16; ++j)
+      for (int j = 0; j < NT; ++j)
         *reinterpret_cast<float2*>(dst + j * 8 + tq * 2) = make_float2(o[j][0] * inv0, o[j][1] * inv0);
       if (tq == 0) p.lse_part[prow + gr] = (l0 > 0.0f) ? (m0 + log2f(l0)) * 0.69314718055994531f : -INFINITY;
     }
-    if (gr + 8 < p.group) {
-      float* dst = p.o_part + (prow + gr + 8) * 128;
+    if (r1) {
+      float* dst = p.o_part + (prow + gr + 8) * D;
 #pragma unroll
-      for (int j = 0; j < 16; ++j)
+      for (int j = 0; j < NT; ++j)
         *reinterpret_cast<float2*>(dst + j * 8 + tq * 2) = make_float2(o[j][2] * inv1, o[j][3] * inv1);
       if (tq == 0) p.lse_part[prow + gr + 8] = (l1 > 0.0f) ? (m1 + log2f(l1)) * 0.69314718055994531f : -INFINITY;
     }
@@ -353,86 +389,114 @@ __global__ void __launch_bounds__(kThreads, 1) decode_split_kernel(const __grid_
   cp_async_wait<0>();
 }
 
-// Merge of the partials of one (request, head) per CTA. The pieces of pair bg
-// come from the warps whose ranges hold its first and last flattened keys and
-// every warp in between with a non-empty range; warp w's piece is in slot
+// Merge of the partials of one (request, head) per CTA. The pieces of triple
+// bg come from the warps whose ranges hold its first and last flattened keys
+// and every warp in between with a non-empty range; warp w's piece is in slot
 // w + bg. The 8 warps take every 8th piece, each keeps an online (max, sum, O)
-// with float4 loads four pieces deep, and the eight results are combined in
+// with vector loads four pieces deep, and the eight results are combined in
 // shared memory. Same formula as the generic merge (LSE weighting, -inf
 // partials weigh 0). This kernel also checks the offsets of its request and
-// records kStatusInternal for offsets that break the contract.
+// records kStatusInternal for offsets that break the contract. It is launched
+// as a programmatic dependent of the split kernel and waits for it first.
 constexpr int kMergeThreads = 256;
 constexpr int kMergeUnroll = 4;
 
-__device__ __forceinline__ void store_row4(__nv_bfloat16* dst, float4 v) {
+template <int VW>
+struct VecF;
+template <>
+struct VecF<4> {
+  using T = float4;
+  static __device__ __forceinline__ T zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+};
+template <>
+struct VecF<2> {
+  using T = float2;
+  static __device__ __forceinline__ T zero() { return make_float2(0.f, 0.f); }
+};
+
+__device__ __forceinline__ float4 vfma(float a, float4 x, float4 y) {
+  return make_float4(fmaf(a, x.x, y.x), fmaf(a, x.y, y.y), fmaf(a, x.z, y.z), fmaf(a, x.w, y.w));
+}
+__device__ __forceinline__ float2 vfma(float a, float2 x, float2 y) { return make_float2(fmaf(a, x.x, y.x), fmaf(a, x.y, y.y)); }
+__device__ __forceinline__ float4 vscale(float a, float4 x) { return make_float4(a * x.x, a * x.y, a * x.z, a * x.w); }
+__device__ __forceinline__ float2 vscale(float a, float2 x) { return make_float2(a * x.x, a * x.y); }
+
+__device__ __forceinline__ void store_vec(__nv_bfloat16* dst, float4 v) {
   uint2 u;
   u.x = pack_bf16x2(v.x, v.y);
   u.y = pack_bf16x2(v.z, v.w);
   *reinterpret_cast<uint2*>(dst) = u;
 }
-__device__ __forceinline__ void store_row4(float* dst, float4 v) { *reinterpret_cast<float4*>(dst) = v; }
+__device__ __forceinline__ void store_vec(__nv_bfloat16* dst, float2 v) {
+  *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(v.x, v.y);
+}
+__device__ __forceinline__ void store_vec(float* dst, float4 v) { *reinterpret_cast<float4*>(dst) = v; }
+__device__ __forceinline__ void store_vec(float* dst, float2 v) { *reinterpret_cast<float2*>(dst) = v; }
 
 // OutT: bf16 for the decoded output, float for a partial (O, LSE) that a
-// later LSE merge combines with other ranks' partials.
-template <typename OutT>
+// later LSE merge combines with other ranks' partials. D/32 floats per lane.
+template <typename OutT, int D>
 __global__ void __launch_bounds__(kMergeThreads, 4) decode_merge_kernel(const __grid_constant__ Params p,
                                                                       OutT* out, float* lse_out) {
+  constexpr int VW = D / 32;
+  using V = typename VecF<VW>::T;
   __shared__ float sm_m[8], sm_l[8];
-  __shared__ float4 sm_o[8][32];
+  __shared__ V sm_o[8][32];
+  wait_primary();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t rh = blockIdx.x;
   const int b = static_cast<int>(rh / p.n_h);
   const int h = static_cast<int>(rh - static_cast<int64_t>(b) * p.n_h);
   const int g = h / p.group;
-  const int hl = h - g * p.group;
-  const int bg = b * p.n_kv + g;
+  const int hr = h - g * p.group;         // head within the group
+  const int u = hr / kUnitRows;           // its unit
+  const int hl = hr - u * kUnitRows;      // its row in the unit's partials
+  const int per_tok = p.n_kv * p.units;
+  const int bg = b * per_tok + g * p.units + u;
   const int64_t o0 = p.offsets[0], oB = p.offsets[p.batch];
   const int64_t base = p.offsets[b], end = p.offsets[b + 1];
   const bool ok = o0 >= 0 && oB >= o0 && oB <= p.kv_rows && base >= o0 && end >= base && end <= oB;
   if (!ok && threadIdx.x == 0) atomicOr(p.status, kStatusInternal);
   const int64_t len = ok ? end - base : 0;
-  const int64_t kt = (oB - o0) * p.n_kv;
+  const int64_t kt = (oB - o0) * per_tok;
   const int64_t W = p.n_warps;
   int64_t w_first = 0, n_pieces = 0;
   if (len > 0) {
-    const int64_t vs = (base - o0) * p.n_kv + g * len;
+    const int64_t vs = (base - o0) * per_tok + static_cast<int64_t>(bg - b * per_tok) * len;
     w_first = range_of(vs, kt, W);
     n_pieces = range_of(vs + len - 1, kt, W) - w_first + 1;
   }
   float m = -INFINITY, l = 0.0f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  V acc = VecF<VW>::zero();
   for (int64_t j0 = warp; j0 < n_pieces; j0 += 8 * kMergeUnroll) {
     // pieces present (a range is empty only when there are fewer keys than ranges)
     uint32_t present = 0;
 #pragma unroll 1
-    for (int u = 0; u < kMergeUnroll; ++u) {
-      const int64_t w = w_first + j0 + u * 8;
-      if (j0 + u * 8 < n_pieces && (kt >= W || range_start(w, kt, W) < range_start(w + 1, kt, W)))
-        present |= 1u << u;
+    for (int uu = 0; uu < kMergeUnroll; ++uu) {
+      const int64_t w = w_first + j0 + uu * 8;
+      if (j0 + uu * 8 < n_pieces && (kt >= W || range_start(w, kt, W) < range_start(w + 1, kt, W)))
+        present |= 1u << uu;
     }
-    float4 x[kMergeUnroll];
+    V x[kMergeUnroll];
     float lj[kMergeUnroll];
 #pragma unroll
-    for (int u = 0; u < kMergeUnroll; ++u) {
-      lj[u] = -INFINITY;
-      x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (present & (1u << u)) {
-        const int64_t row = (w_first + j0 + u * 8 + bg) * p.group + hl;
-        lj[u] = __ldcs(p.lse_part + row);
-        x[u] = __ldcs(reinterpret_cast<const float4*>(p.o_part + row * 128) + lane);
+    for (int uu = 0; uu < kMergeUnroll; ++uu) {
+      lj[uu] = -INFINITY;
+      x[uu] = VecF<VW>::zero();
+      if (present & (1u << uu)) {
+        const int64_t row = (w_first + j0 + uu * 8 + bg) * p.rows + hl;
+        lj[uu] = __ldcs(p.lse_part + row);
+        x[uu] = __ldcs(reinterpret_cast<const V*>(p.o_part + row * D) + lane);
       }
     }
 #pragma unroll
-    for (int u = 0; u < kMergeUnroll; ++u) {
-      if (lj[u] == -INFINITY) continue;
-      const float m_new = fmaxf(m, lj[u]);
+    for (int uu = 0; uu < kMergeUnroll; ++uu) {
+      if (lj[uu] == -INFINITY) continue;   // a part at -inf weighs 0 and its O is not read
+      const float m_new = fmaxf(m, lj[uu]);
       const float so = __expf(m - m_new);   // 0 when m was -inf
-      const float wj = __expf(lj[u] - m_new);
+      const float wj = __expf(lj[uu] - m_new);
       l = l * so + wj;
-      acc.x = fmaf(wj, x[u].x, acc.x * so);
-      acc.y = fmaf(wj, x[u].y, acc.y * so);
-      acc.z = fmaf(wj, x[u].z, acc.z * so);
-      acc.w = fmaf(wj, x[u].w, acc.w * so);
+      acc = vfma(wj, x[uu], vscale(so, acc));
       m = m_new;
     }
   }
@@ -447,21 +511,18 @@ __global__ void __launch_bounds__(kMergeThreads, 4) decode_merge_kernel(const __
 #pragma unroll
     for (int w = 0; w < 8; ++w) M = fmaxf(M, sm_m[w]);
     float L = 0.0f;
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    V o = VecF<VW>::zero();
     if (M != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < 8; ++w) {
-        const float sc = expf(sm_m[w] - M);   // 0 for warps that saw no piece
+        if (sm_m[w] == -INFINITY) continue;   // a warp that saw no piece
+        const float sc = expf(sm_m[w] - M);
         L += sm_l[w] * sc;
-        const float4 a = sm_o[w][lane];
-        o.x = fmaf(sc, a.x, o.x);
-        o.y = fmaf(sc, a.y, o.y);
-        o.z = fmaf(sc, a.z, o.z);
-        o.w = fmaf(sc, a.w, o.w);
+        o = vfma(sc, sm_o[w][lane], o);
       }
     }
     const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
-    store_row4(out + rh * 128 + lane * 4, make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv));
+    store_vec(out + rh * D + lane * VW, vscale(inv, o));
     if (lse_out && lane == 0) lse_out[rh] = (L > 0.0f) ? M + logf(L) : -INFINITY;
   }
 }

@@ -35,9 +35,10 @@ __device__ __forceinline__ void store4(__nv_bfloat16* dst, float4 v) {
   *reinterpret_cast<uint2*>(dst) = u;
 }
 
+// o_parts / lse_parts carry no __restrict__: out and lse_out may alias part 0.
 template <typename OutT, int R>
-__global__ void __launch_bounds__(kThreads, R <= 2 ? 3 : 2) merge_kernel(const float* __restrict__ o_parts,
-                                                          const float* __restrict__ lse_parts, int n_parts,
+__global__ void __launch_bounds__(kThreads, R <= 2 ? 3 : 2) merge_kernel(const float* o_parts,
+                                                          const float* lse_parts, int n_parts,
                                                           int64_t o_stride, int64_t l_stride, int64_t n_rowheads,
                                                           int d, OutT* out, float* lse_out) {
   constexpr int C = kLoads / R;
@@ -91,12 +92,15 @@ __global__ void __launch_bounds__(kThreads, R <= 2 ? 3 : 2) merge_kernel(const f
           acc[r].w *= sc;
 #pragma unroll
           for (int c = 0; c < C; ++c) {
-            const float w = expf(lj[r][c] - mu);
+            // a part at -inf weighs 0: its O row is not used (it may hold anything)
+            const bool used = lj[r][c] != -INFINITY;
+            const float w = used ? expf(lj[r][c] - mu) : 0.0f;
+            const float4 xv = used ? x[r][c] : make_float4(0.f, 0.f, 0.f, 0.f);
             l[r] += w;
-            acc[r].x = fmaf(w, x[r][c].x, acc[r].x);
-            acc[r].y = fmaf(w, x[r][c].y, acc[r].y);
-            acc[r].z = fmaf(w, x[r][c].z, acc[r].z);
-            acc[r].w = fmaf(w, x[r][c].w, acc[r].w);
+            acc[r].x = fmaf(w, xv.x, acc[r].x);
+            acc[r].y = fmaf(w, xv.y, acc[r].y);
+            acc[r].z = fmaf(w, xv.z, acc[r].z);
+            acc[r].w = fmaf(w, xv.w, acc[r].w);
           }
           m[r] = m_new;
         }

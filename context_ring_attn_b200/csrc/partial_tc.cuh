@@ -523,7 +523,7 @@ __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Para
           float r[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(o[i]) * wb;
-          if (p.accumulate) {
+          if (p.accumulate && wa != 0.0f) {   // an earlier row at -inf weighs 0 and is not read
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
               const float4 pv = *reinterpret_cast<const float4*>(dst + c * 32 + i);

@@ -98,10 +98,17 @@ int32_t cp_abi_version(void) { return CP_ABI_VERSION; }
 
 cp_status cp_shard_plan(const cp_segment* segs, int32_t n_seg, int32_t n_ranks,
                         cp_shard_mode mode, int64_t* chunk_bounds, int64_t* rank_rows,
-                        int64_t* token_index) {
+                        int64_t* token_index, int64_t* sizes_out) {
   if (n_ranks < 1 || !segs_ok(segs, n_seg)) return CP_ERR_INVALID_ARG;
   if (mode != CP_SHARD_LOAD_BALANCED && mode != CP_SHARD_CONTIGUOUS) return CP_ERR_INVALID_ARG;
   const int64_t n_chunks = 2 * static_cast<int64_t>(n_ranks);
+  if (sizes_out) {
+    int64_t tokens = 0;
+    for (int32_t s = 0; s < n_seg; ++s) tokens += segs[s].len;
+    sizes_out[0] = static_cast<int64_t>(n_seg) * (n_chunks + 1);
+    sizes_out[1] = static_cast<int64_t>(n_ranks) + 1;
+    sizes_out[2] = tokens;
+  }
   if (chunk_bounds) {
     for (int32_t s = 0; s < n_seg; ++s)
       for (int64_t c = 0; c <= n_chunks; ++c)

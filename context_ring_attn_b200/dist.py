@@ -12,6 +12,13 @@ chunks i and 2N-1-i of every segment; or contiguous).
   every Q shard that reaches it to its local KV, then an all-to-all returns
   the partials to the owners of the queries, which merge them.
 
+* CP groups per KV head (section 5, key implementation details, item 1: one
+  CP communication group per KV head): with the heads split across G groups
+  of ranks (a KV head and the query heads that share it per group, as tensor
+  parallelism splits them), each group runs its own ring over its heads'
+  slices; kv_head_groups() forms the groups and head_slices() names each
+  group's heads.
+
 This module is plumbing: torch.distributed moves the shards (NCCL between
 GPUs, point-to-point sends into a local buffer; no remote loads); the
 attention and the merge are the library's kernels (cp_attn_partial,
@@ -36,6 +43,34 @@ class Segment:
     row0: int
     pos0: int
     seq: int = 0
+
+
+def kv_head_groups(n_groups: int):
+    """Split the world into `n_groups` CP rings of world/n_groups consecutive
+    ranks each: ring i serves KV-head group i. Every rank must call this (each
+    group is created collectively, in the same order on all ranks). Returns
+    (this rank's process group, its group index)."""
+    world, rank = dist.get_world_size(), dist.get_rank()
+    if n_groups < 1 or world % n_groups:
+        raise ValueError(f"world size {world} is not a multiple of {n_groups} KV-head groups")
+    cp = world // n_groups
+    mine = None
+    for i in range(n_groups):
+        g = dist.new_group(list(range(i * cp, (i + 1) * cp)))
+        if rank // cp == i:
+            mine = g
+    return mine, rank // cp
+
+
+def head_slices(n_h: int, n_kv: int, n_groups: int, index: int):
+    """Query-head and KV-head slices of KV-head group `index`: n_kv/n_groups
+    consecutive KV heads and the n_h/n_kv query heads of each (GQA: query head
+    h uses KV head floor(h / (n_h/n_kv)))."""
+    if n_h % n_kv or n_kv % n_groups:
+        raise ValueError("n_kv must be a multiple of the group count and n_h of n_kv")
+    kv_per = n_kv // n_groups
+    g = n_h // n_kv
+    return slice(index * kv_per * g, (index + 1) * kv_per * g), slice(index * kv_per, (index + 1) * kv_per)
 
 
 def _local(ranges, base: int = 0):

@@ -59,6 +59,12 @@ class RingSchedule:
         return sum(B.cp_block_pairs(self.ranges, self.blocks[i], causal) for i in range(self.n_ranks ** 2))
 
 
+def _nvtx(name: str):
+    """An NVTX range (visible in an Nsight Systems timeline) around one host
+    step of a schedule: each ring step's launch and each merge."""
+    return torch.cuda.nvtx.range(name)
+
+
 def partial_buffers(q_rows: int, n_h: int, d: int, n_parts: int, device="cuda"):
     o = torch.empty((n_parts * q_rows, n_h, d), dtype=torch.float32, device=device)
     lse = torch.empty((n_parts * q_rows, n_h), dtype=torch.float32, device=device)
@@ -88,33 +94,39 @@ def run_ring(sched: RingSchedule, q, k, v, n_h: int, n_kv: int, out, lse_out=Non
     if workspace is None:
         workspace = torch.zeros(B.cp_workspace_size(B.CP_OP_PARTIAL, 0, n_h, d, 1), dtype=torch.uint8,
                                 device=q.device)
+    if merge not in ("fused", "final", "running"):
+        raise ValueError(merge)
     if merge == "fused":
         lse_acc = lse_out if lse_out is not None else lse_parts
         for t in range(n):
             blocks = sched.step_blocks(t, q_rows, part_of=lambda _p: 0)
-            B.cp_attn_partial_fused(q, k, v, n_h, n_kv, scale, causal, sched.ranges, sched.n_ranges, blocks, n,
-                                    o_parts, lse_acc, t > 0, out if t == n - 1 else None, workspace, stream)
+            with _nvtx(f"ring step {t} (fused merge)"):
+                B.cp_attn_partial_fused(q, k, v, n_h, n_kv, scale, causal, sched.ranges, sched.n_ranges, blocks, n,
+                                        o_parts, lse_acc, t > 0, out if t == n - 1 else None, workspace, stream)
         return out
     if merge == "final":
         for t in range(n):
             blocks = sched.step_blocks(t, q_rows)
-            B.cp_attn_partial(q, k, v, n_h, n_kv, scale, causal, sched.ranges, sched.n_ranges, blocks, n,
-                              o_parts, lse_parts, workspace, stream)
-        B.cp_attn_merge(o_parts, lse_parts, n, q_rows, q_rows, n_h, d, out, lse_out, stream)
-    elif merge == "running":
+            with _nvtx(f"ring step {t}"):
+                B.cp_attn_partial(q, k, v, n_h, n_kv, scale, causal, sched.ranges, sched.n_ranges, blocks, n,
+                                  o_parts, lse_parts, workspace, stream)
+        with _nvtx(f"merge {n}-way"):
+            B.cp_attn_merge(o_parts, lse_parts, n, q_rows, q_rows, n_h, d, out, lse_out, stream)
+    else:
         for t in range(n):
             target = 0 if t == 0 else 1
             blocks = sched.step_blocks(t, q_rows, part_of=lambda _p, _t=target: _t)
-            B.cp_attn_partial(q, k, v, n_h, n_kv, scale, causal, sched.ranges, sched.n_ranges, blocks, n,
-                              o_parts, lse_parts, workspace, stream)
+            with _nvtx(f"ring step {t}"):
+                B.cp_attn_partial(q, k, v, n_h, n_kv, scale, causal, sched.ranges, sched.n_ranges, blocks, n,
+                                  o_parts, lse_parts, workspace, stream)
             if t == 0 and n > 1:
                 continue
-            if t == n - 1:
-                B.cp_attn_merge(o_parts, lse_parts, 2 if n > 1 else 1, q_rows, q_rows, n_h, d, out, lse_out, stream)
-            else:
-                B.cp_attn_merge(o_parts, lse_parts, 2, q_rows, q_rows, n_h, d, o_parts, lse_parts, stream)
-    else:
-        raise ValueError(merge)
+            with _nvtx("merge running"):
+                if t == n - 1:
+                    B.cp_attn_merge(o_parts, lse_parts, 2 if n > 1 else 1, q_rows, q_rows, n_h, d, out, lse_out,
+                                    stream)
+                else:
+                    B.cp_attn_merge(o_parts, lse_parts, 2, q_rows, q_rows, n_h, d, o_parts, lse_parts, stream)
     return out
 
 
@@ -176,6 +188,8 @@ class DecodeCP:
         """q_ranks: the queries as every rank holds them, [N*B, n_h, d] (q repeated
         N times, rank-major). out [B, n_h, d] bf16, lse_out [B, n_h] fp32."""
         n_h, d = int(q_ranks.shape[1]), int(q_ranks.shape[2])
-        B.cp_decode_partial(q_ranks, self.k, self.v, self.offsets, n_h, n_kv, n_splits, softmax_scale,
-                            o_parts, lse_parts, workspace, stream)
-        B.cp_attn_merge(o_parts, lse_parts, self.n_ranks, self.n_req, self.n_req, n_h, d, out, lse_out, stream)
+        with _nvtx("cp decode: rank partials"):
+            B.cp_decode_partial(q_ranks, self.k, self.v, self.offsets, n_h, n_kv, n_splits, softmax_scale,
+                                o_parts, lse_parts, workspace, stream)
+        with _nvtx("cp decode: merge"):
+            B.cp_attn_merge(o_parts, lse_parts, self.n_ranks, self.n_req, self.n_req, n_h, d, out, lse_out, stream)

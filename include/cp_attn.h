@@ -36,7 +36,7 @@
 extern "C" {
 #endif
 
-#define CP_ABI_VERSION 1
+#define CP_ABI_VERSION 2
 
 typedef enum {
   CP_OK = 0,
@@ -112,11 +112,14 @@ int32_t cp_abi_version(void);
  *  rank_rows    [N+1]: prefix offsets of each rank's rows in token_index.
  *  token_index  [sum of len]: buffer rows held by rank 0, then rank 1, ...;
  *                per rank, segment by segment, chunks in ascending order.
+ *  sizes_out    [3]: the element counts of the three arrays above,
+ *                n_seg*(2N+1), N+1 and sum of len, so that a caller can call
+ *                once with NULL arrays to size them, then again to fill them.
  * Any output pointer may be NULL to skip it. Errors: CP_ERR_INVALID_ARG for
  * n_ranks < 1, n_seg < 0, a negative len/row0/pos0 or a nonzero reserved field. */
 cp_status cp_shard_plan(const cp_segment* segs, int32_t n_seg, int32_t n_ranks,
                         cp_shard_mode mode, int64_t* chunk_bounds, int64_t* rank_rows,
-                        int64_t* token_index);
+                        int64_t* token_index, int64_t* sizes_out);
 
 /* The ranges rank `rank` holds: for each segment in order, its two chunks in
  * ascending chunk order, empty chunks left out. `out` holds up to 2*n_seg
@@ -264,24 +267,29 @@ cp_status cp_attn_merge(const float* o_parts, const float* lse_parts, int32_t n_
 /* Split-KV decode (Flash Decoding; method page, section 5 software stack).
  * Request b has one query row q[b] at position L_b - 1 and keys k/v rows
  * kv_offsets[b] .. kv_offsets[b+1]-1 (L_b = difference), all visible.
- * The splits are cut over the whole batch rather than per request: the keys
- * of every (request, KV head) pair, in order, form one sequence of
- * Kt = n_kv*(kv_offsets[batch] - kv_offsets[0]) keys, cut into W equal ranges,
- * W = 8*min(SM count, ceil(n_splits*batch*n_kv/8)). So n_splits caps the
- * average number of splits per pair, and every range holds the same number
- * of keys whatever the mix of lengths. Each range leaves one partial per pair
- * it overlaps in the workspace; the partials of each (request, head) are then
- * merged as in cp_attn_merge. The result does not depend on the cut beyond
- * rounding.
+ * The query heads of a KV head (G = n_h/n_kv of them, GQA) are taken 16 at a
+ * time: G <= 16 is one unit, G = 16u is u units. The splits are cut over the
+ * whole batch rather than per request: the keys of every (request, KV head,
+ * unit) triple, in order, form one sequence of
+ * Kt = n_kv*U*(kv_offsets[batch] - kv_offsets[0]) keys (U units per KV head),
+ * cut into W equal ranges, W = 8*min(SM count, ceil(n_splits*batch*n_kv*U/8)).
+ * So n_splits caps the average number of splits per triple, and every range
+ * holds the same number of keys whatever the mix of lengths. Each range leaves
+ * one partial per triple it overlaps in the workspace; the partials of each
+ * (request, head) are then merged as in cp_attn_merge (a second launch that
+ * starts as a programmatic dependent of the first). The result does not
+ * depend on the cut beyond rounding.
  *   q [batch, n_h, d] bf16; k, v [kv_rows, n_kv, d] bf16;
  *   kv_offsets: DEVICE int64 [batch+1], non-decreasing, last <= kv_rows
  *   (with offsets that break this no K/V row outside [0, kv_rows) is read,
  *   and cp_check_status then reports CP_ERR_INTERNAL);
  *   out [batch, n_h, d] bf16; lse_out [batch, n_h] fp32 (may be NULL).
- * Supports dtype CP_BF16, d == 128, n_h/n_kv in {1, 2, 4, 8, 16},
- * 1 <= n_splits <= 1024, Kt*W < 2^53.
- * A request with L_b = 0 yields out = 0, lse = -inf.
- * workspace: >= cp_workspace_size(CP_OP_DECODE, batch, n_h, d, n_splits). */
+ * Supports dtype CP_BF16, d in {64, 128}, a group G = n_h/n_kv <= 16 or a
+ * multiple of 16 up to 128 (CP_ERR_UNSUPPORTED otherwise), 1 <= n_splits <=
+ * 1024, kv_rows*n_kv*U*(W+1) < 2^53. Every argument is checked before
+ * anything is launched. A request with L_b = 0 yields out = 0, lse = -inf.
+ * workspace: >= cp_workspace_size(CP_OP_DECODE, batch, n_h, d, n_splits),
+ * 256-byte aligned, status word zeroed (cp_reset_status). */
 cp_status cp_decode(const void* q, const void* k, const void* v, cp_dtype dtype,
                     const int64_t* kv_offsets, int32_t batch, int64_t kv_rows, int32_t n_h,
                     int32_t n_kv, int32_t d, int32_t n_splits, float softmax_scale, void* out,
@@ -308,23 +316,34 @@ cp_status cp_decode_partial(const void* q, const void* k, const void* v, cp_dtyp
  * start-up). The method's pages have no counterpart to this entry point.
  *
  * Same arguments, results and limits as cp_decode, without the workspace: the
- * split partials live in a fixed 32 MiB array in the library's device memory,
- * which every GPU that loads the library holds until the process exits.
- *  - Requests whose partials, (W + batch*n_kv)*(n_h/n_kv) rows of d+1 floats
- *    with W as in cp_decode for the current device, need more than the array
- *    are rejected with CP_ERR_WORKSPACE before any launch.
+ * split partials and the status word live in a fixed 32 MiB array in the
+ * library's device memory, which every GPU that loads the library holds until
+ * the process exits.
+ *  - Every argument is checked first; a call that returns an error has
+ *    enqueued nothing. Requests whose partials, (W + batch*n_kv*U)*min(G, 16)
+ *    rows of d+1 floats with W and U as in cp_decode for the current device,
+ *    need more than the array are rejected with CP_ERR_WORKSPACE.
  *  - The first call on a device looks up the array's device address for that
  *    device (the device current at the call); make that first call before any
  *    stream capture.
  *  - Every call shares the one array, which keeps the last call's contents;
- *    each call clears the status word it needs and rewrites every partial it
- *    reads. Calls that overlap on the GPU (different streams without
- *    ordering, or several host threads) race on the array.
+ *    each call clears the status word (stream-ordered) and rewrites every
+ *    partial it reads. Calls that overlap on the GPU (different streams
+ *    without ordering, or several host threads) race on the array.
+ *  - Device-side failures of a call (offsets that break the contract) are
+ *    reported by cp_decode_static_status until the next call clears them.
  *  - Nothing is allocated or freed. */
 cp_status cp_decode_static(const void* q, const void* k, const void* v, cp_dtype dtype,
                            const int64_t* kv_offsets, int32_t batch, int64_t kv_rows, int32_t n_h,
                            int32_t n_kv, int32_t d, int32_t n_splits, float softmax_scale, void* out,
                            float* lse_out, void* cuda_stream);
+
+/* The device-side status of the latest cp_decode_static call on the current
+ * device (the counterpart of cp_check_status for the fixed array):
+ * synchronises `cuda_stream` (pass the stream that call used), then returns
+ * CP_OK, CP_ERR_INTERNAL (offsets that break the contract) or CP_ERR_TIMEOUT.
+ * Allocates nothing. */
+cp_status cp_decode_static_status(void* cuda_stream);
 
 #ifdef __cplusplus
 }

@@ -51,3 +51,18 @@ def sample_rows(rng, n_rows: int, n_sample: int, must=()) -> np.ndarray:
     must = np.unique(np.asarray([m for m in must if 0 <= m < n_rows], dtype=np.int64))
     rest = rng.choice(n_rows, size=min(n_rows, max(0, n_sample - must.size)), replace=False)
     return np.unique(np.concatenate([must, rest]))
+
+
+def oracle_rows(fn, n_rows: int, chunk: int = 128, workers: int | None = None):
+    """Run fn(lo, hi) -> (O, LSE) of rows lo..hi-1 of a sample on a thread
+    pool (numpy's BLAS and ufunc loops release the GIL) and stack the results
+    in row order. Only the reference runs here; it is called unchanged, on
+    slices of the sampled rows."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    bounds = [(lo, min(n_rows, lo + chunk)) for lo in range(0, n_rows, chunk)]
+    workers = workers or max(1, min(16, os.cpu_count() or 1))
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        parts = list(ex.map(lambda b: fn(*b), bounds))
+    return np.concatenate([x[0] for x in parts]), np.concatenate([x[1] for x in parts])

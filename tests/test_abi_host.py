@@ -33,7 +33,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_version_and_strings(L):
-    assert B.cp_abi_version() == 1
+    assert B.cp_abi_version() == 2
     for code in range(7):
         assert B.status_string(code)
     assert "unknown" in B.status_string(99)
@@ -114,9 +114,9 @@ def test_merge_and_decode_reject_bad_arguments(L):
     assert dec(off=None) == B.CP_ERR_INVALID_ARG
     assert dec(splits=0) == B.CP_ERR_UNSUPPORTED
     assert dec(splits=5000) == B.CP_ERR_UNSUPPORTED
-    assert dec(n_h=48, n_kv=1) == B.CP_ERR_UNSUPPORTED
-    assert dec(n_h=24, n_kv=2) == B.CP_ERR_UNSUPPORTED   # group 12 does not divide 16
-    assert dec(d=64) == B.CP_ERR_UNSUPPORTED
+    assert dec(n_h=40, n_kv=1) == B.CP_ERR_UNSUPPORTED   # a group above 16 must be a multiple of 16
+    assert dec(n_h=256, n_kv=1) == B.CP_ERR_UNSUPPORTED  # groups above 128
+    assert dec(d=96) == B.CP_ERR_UNSUPPORTED
     assert dec(dtype=B.CP_F32) == B.CP_ERR_UNSUPPORTED
     assert dec(ws_bytes=1024) == B.CP_ERR_WORKSPACE
     assert dec(ws=None) == B.CP_ERR_WORKSPACE
@@ -131,7 +131,7 @@ def test_planning_rejects_bad_arguments(L):
     assert L.cp_rank_ranges(segs, 1, 2, 0, 2, out, ctypes.byref(n)) == B.CP_ERR_INVALID_ARG
     assert L.cp_rank_ranges(segs, 1, 2, 9, 0, out, ctypes.byref(n)) == B.CP_ERR_INVALID_ARG
     bad = B.segments([(-1, 0, 0, 0)])
-    assert L.cp_shard_plan(bad, 1, 2, 0, None, None, None) == B.CP_ERR_INVALID_ARG
+    assert L.cp_shard_plan(bad, 1, 2, 0, None, None, None, None) == B.CP_ERR_INVALID_ARG
     ranges = (B.cp_range * 2)()
     blocks = (B.cp_block * 4)()
     assert L.cp_ring_schedule(segs, 1, segs, 1, 2, 0, 0, ranges, 2, ctypes.byref(n), blocks, None) == \
@@ -164,3 +164,38 @@ def test_pair_kernel_build_compiles_and_exports(tmp_path):
     lib = ctypes.CDLL(out)
     for n in header_functions():
         assert hasattr(lib, n), n
+
+
+def test_decode_takes_every_listed_shape(L):
+    """Head dims 64 and 128 and every GQA group up to 128 heads that the
+    boundary lists get past the shape checks (the call then stops at the
+    missing workspace, before any CUDA call)."""
+    for d in (64, 128):
+        for n_h, n_kv in ((16, 1), (16, 16), (12, 4), (8, 1), (32, 1), (64, 4), (128, 8), (128, 1), (64, 2)):
+            for fn in ("cp_decode", "cp_decode_partial"):
+                code = getattr(L, fn)(FAKE, FAKE, FAKE, B.CP_BF16, FAKE, 4, 100, n_h, n_kv, d, 256, 0.1, FAKE, FAKE,
+                                      FAKE, 0, None)
+                assert code == B.CP_ERR_WORKSPACE, (fn, d, n_h, n_kv, code)
+
+
+def test_decode_static_checks_arguments_on_the_host(L):
+    """Rejected before any CUDA call (this test runs without a GPU)."""
+    def st(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, dtype=B.CP_BF16, off=FAKE, batch=4, kv_rows=100, n_h=16, n_kv=1, d=128,
+                 splits=256, scale=0.1, out=FAKE, lse=FAKE)
+        a.update(kw)
+        return L.cp_decode_static(a["q"], a["k"], a["v"], a["dtype"], a["off"], a["batch"], a["kv_rows"], a["n_h"],
+                                  a["n_kv"], a["d"], a["splits"], a["scale"], a["out"], a["lse"], None)
+    assert st(q=None) == B.CP_ERR_INVALID_ARG
+    assert st(d=96) == B.CP_ERR_UNSUPPORTED
+    assert st(n_h=40) == B.CP_ERR_UNSUPPORTED
+    assert st(splits=0) == B.CP_ERR_UNSUPPORTED
+    assert st(scale=float("inf")) == B.CP_ERR_INVALID_ARG
+    assert st(k=FAKE + 8) == B.CP_ERR_INVALID_ARG
+
+
+def test_shard_plan_sizes_query(L):
+    segs = B.segments([(10, 0, 0, 0), (7, 10, 0, 1)])
+    sz = (ctypes.c_int64 * 3)()
+    assert L.cp_shard_plan(segs, 2, 3, 0, None, None, None, sz) == B.CP_OK
+    assert list(sz) == [2 * 7, 4, 17]

@@ -17,14 +17,19 @@ import numpy as np
 import pytest
 
 CASES = [
-    # (name, world, variant, mode)
-    ("prefill", 2, "kv", "lb"),
-    ("prefill", 4, "kv", "lb"),
-    ("prefill", 4, "q", "lb"),
-    ("prefill", 2, "q", "contig"),
-    ("varlen", 4, "kv", "contig"),
-    ("persistent", 4, "q", "lb"),
-    ("persistent", 2, "kv", "lb"),
+    # (name, world, variant, mode, KV-head groups)
+    ("prefill", 2, "kv", "lb", 1),
+    ("prefill", 4, "kv", "lb", 1),
+    ("prefill", 4, "q", "lb", 1),
+    ("prefill", 2, "q", "contig", 1),
+    ("varlen", 4, "kv", "contig", 1),
+    ("persistent", 4, "q", "lb", 1),
+    ("persistent", 2, "kv", "lb", 1),
+    # one CP ring per KV head: world 4 = 2 KV heads x a ring of 2
+    ("prefill", 4, "kv", "lb", 2),
+    ("prefill", 4, "q", "lb", 2),
+    ("persistent", 4, "q", "lb", 2),
+    ("varlen", 4, "kv", "lb", 2),
 ]
 
 
@@ -92,12 +97,12 @@ def _problem(name):
     return q_segs, kv_segs, q_pos, k_pos, q_seq, k_seq, tq, tk
 
 
-def _worker(rank, world, port, name, variant, mode, out_dir):
+def _worker(rank, world, port, name, variant, mode, groups, out_dir):
     try:
         import torch
         import torch.distributed as dist
         from context_ring_attn_b200 import binding as B
-        from context_ring_attn_b200.dist import RingAttention
+        from context_ring_attn_b200.dist import RingAttention, head_slices, kv_head_groups
         from oracle import attention as OA
 
         dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
@@ -109,12 +114,17 @@ def _worker(rank, world, port, name, variant, mode, out_dir):
         k = rng.standard_normal((tk, n_kv, d))
         v = rng.standard_normal((tk, n_kv, d))
         scale = 1.0 / np.sqrt(d)
-        ra = RingAttention(q_segs, kv_segs, n_h, n_kv, d,
+        group, gi = (None, 0) if groups == 1 else kv_head_groups(groups)
+        hq, hk = head_slices(n_h, n_kv, groups, gi)
+        q, k, v = q[:, hq], k[:, hk], v[:, hk]   # this ring's heads
+        ra = RingAttention(q_segs, kv_segs, n_h // groups, n_kv // groups, d,
                            B.CP_PASS_KV if variant == "kv" else B.CP_PASS_Q,
-                           B.CP_SHARD_LOAD_BALANCED if mode == "lb" else B.CP_SHARD_CONTIGUOUS,
+                           B.CP_SHARD_LOAD_BALANCED if mode == "lb" else B.CP_SHARD_CONTIGUOUS, group=group,
                            partial_fn=_oracle_partial, merge_fn=_oracle_merge)
+        assert ra.n == world // groups
         qi, ki = ra.q_shard_rows().numpy(), ra.kv_shard_rows().numpy()
         out, lse = ra.forward(torch.from_numpy(q[qi]), torch.from_numpy(k[ki]), torch.from_numpy(v[ki]), scale)
+        # the unsharded attention of these rows, restricted to this ring's heads
         o_ref, l_ref = OA.attention(q[qi], k, v, q_pos[qi], k_pos, q_seq[qi], k_seq, scale)
         err = float(np.abs(out.numpy() - o_ref).max(initial=0.0))
         fin = np.isfinite(l_ref)
@@ -123,7 +133,7 @@ def _worker(rank, world, port, name, variant, mode, out_dir):
         # every row of Q is owned by exactly one rank
         owned = torch.zeros(tq, dtype=torch.int64)
         owned[torch.from_numpy(qi)] += 1
-        dist.all_reduce(owned)
+        dist.all_reduce(owned, group=group)
         dist.destroy_process_group()
         with open(os.path.join(out_dir, f"r{rank}"), "w") as f:
             f.write(f"{err} {lerr} {int(same_inf)} {int(bool((owned == 1).all()))}\n")
@@ -132,12 +142,12 @@ def _worker(rank, world, port, name, variant, mode, out_dir):
             f.write("EXC " + traceback.format_exc().replace("\n", " | "))
 
 
-@pytest.mark.parametrize("name,world,variant,mode", CASES)
-def test_ring_over_gloo_matches_unsharded_attention(name, world, variant, mode):
+@pytest.mark.parametrize("name,world,variant,mode,groups", CASES)
+def test_ring_over_gloo_matches_unsharded_attention(name, world, variant, mode, groups):
     ctx = mp.get_context("spawn")
     port = _free_port()
     with tempfile.TemporaryDirectory() as tmp:
-        procs = [ctx.Process(target=_worker, args=(r, world, port, name, variant, mode, tmp)) for r in range(world)]
+        procs = [ctx.Process(target=_worker, args=(r, world, port, name, variant, mode, groups, tmp)) for r in range(world)]
         for p in procs:
             p.start()
         for p in procs:

@@ -181,18 +181,62 @@ def test_merge_in_place():
     check(od[0].cpu().numpy(), ld[0].cpu().numpy(), o_ref, l_ref, "f32")
 
 
+@pytest.mark.parametrize("n_parts", [2, 3, 8])
+def test_merge_ignores_rows_of_parts_at_minus_inf(n_parts):
+    """A part whose LSE is -inf weighs 0, so whatever its O row holds (NaN
+    here) must not reach the output."""
+    rng = np.random.default_rng(100 + n_parts)
+    rows, n_h, d = 29, 4, 128
+    o = rng.standard_normal((n_parts, rows, n_h, d)).astype(np.float32)
+    lse = rng.standard_normal((n_parts, rows, n_h)).astype(np.float32)
+    lse[0, ::3] = -np.inf
+    lse[:, 7, 2] = -np.inf          # every part empty: O = 0, LSE = -inf
+    o_clean = np.where(np.isinf(lse)[..., None], 0.0, o).astype(np.float32)
+    o_ref, l_ref = OA.merge(list(o_clean), list(lse))
+    o_dirty = np.where(np.isinf(lse)[..., None], np.nan, o).astype(np.float32)
+    out = torch.empty((rows, n_h, d), dtype=torch.float32, device="cuda")
+    lse_out = torch.empty((rows, n_h), dtype=torch.float32, device="cuda")
+    B.cp_attn_merge(dev(o_dirty, "f32"), dev(lse, "f32"), n_parts, rows, rows, n_h, d, out, lse_out)
+    torch.cuda.synchronize()
+    check(out.cpu().numpy(), lse_out.cpu().numpy(), o_ref, l_ref, "f32", "merge with NaN in -inf parts")
+
+
+def test_fused_accumulate_ignores_earlier_rows_at_minus_inf():
+    """cp_attn_partial_fused with accumulate: an earlier (O, LSE) at -inf weighs
+    0, so a NaN O row there must not reach the merged row."""
+    t, n_h, n_kv, d = 300, 16, 1, 128
+    pr = synth.make_prefill(t, n_h, n_kv, d, "bf16", 321, 0.5)
+    q, k, v = dev(pr.q_raw, "bf16"), dev(pr.k_raw, "bf16"), dev(pr.v_raw, "bf16")
+    ranges = (B.cp_range * 2)(B.cp_range(0, 0, t, 0, 0), B.cp_range(0, 0, t, 0, 0))
+    blocks = (B.cp_block * 1)(B.cp_block(0, 1, 1, 1, 0))
+    o_acc = torch.full((t, n_h, d), float("nan"), dtype=torch.float32, device="cuda")
+    lse_acc = torch.full((t, n_h), float("-inf"), dtype=torch.float32, device="cuda")
+    out = torch.empty((t, n_h, d), dtype=torch.bfloat16, device="cuda")
+    B.cp_attn_partial_fused(q, k, v, n_h, n_kv, 1 / math.sqrt(d), True, ranges, 2, blocks, 1, o_acc, lse_acc, True,
+                            out, _ws())
+    torch.cuda.synchronize()
+    o_ref, l_ref = OA.attention(pr.q, pr.k, pr.v, np.arange(t), np.arange(t))
+    check(out.float().cpu().numpy(), lse_acc.cpu().numpy(), o_ref, l_ref, "bf16", "fused accumulate over -inf rows")
+
+
 # ---------------------------------------------------------------------------- decode
-@pytest.mark.parametrize("n_h,n_kv,n_splits", [(16, 1, 256), (16, 2, 16), (16, 1, 1), (64, 4, 256)])
-def test_decode(n_h, n_kv, n_splits):
+@pytest.mark.parametrize("n_h,n_kv,n_splits,d", [
+    (16, 1, 256, 128), (16, 2, 16, 128), (16, 1, 1, 128), (64, 4, 256, 128),
+    (12, 4, 32, 128),     # G = 3: rows past the group are zero
+    (128, 1, 64, 128),    # MQA, G = 128: eight 16-head units per KV head
+    (64, 2, 16, 128),     # G = 32 on two KV heads
+    (16, 1, 256, 64), (8, 8, 16, 64), (128, 2, 64, 64),   # head dim 64
+])
+def test_decode(n_h, n_kv, n_splits, d):
     lens = [0, 5, 100, 255, 256, 1000, 3001, 64]
-    dc = synth.make_decode(len(lens), n_h, n_kv, 128, lens, 40 + n_splits, 0.5)
+    dc = synth.make_decode(len(lens), n_h, n_kv, d, lens, 40 + n_splits + n_h + d, 0.5)
     q, k, v = dev(dc.q_raw, "bf16"), dev(dc.k_raw, "bf16"), dev(dc.v_raw, "bf16")
     off = torch.from_numpy(dc.offsets).cuda()
-    out = torch.empty((len(lens), n_h, 128), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((len(lens), n_h, d), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((len(lens), n_h), dtype=torch.float32, device="cuda")
-    ws = torch.zeros(B.cp_workspace_size(B.CP_OP_DECODE, len(lens), n_h, 128, n_splits), dtype=torch.uint8,
+    ws = torch.zeros(B.cp_workspace_size(B.CP_OP_DECODE, len(lens), n_h, d, n_splits), dtype=torch.uint8,
                      device="cuda")
-    B.cp_decode(q, k, v, off, n_h, n_kv, n_splits, 1 / math.sqrt(128), out, lse, ws)
+    B.cp_decode(q, k, v, off, n_h, n_kv, n_splits, 1 / math.sqrt(d), out, lse, ws)
     B.cp_check_status(ws)
     o_ref, l_ref = OD.decode(dc.q, dc.k, dc.v, dc.offsets)
     check(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "bf16", "decode")
@@ -220,13 +264,16 @@ def _decode_case(lens, n_h, n_kv, seed):
     return dc, dev(dc.q_raw, "bf16"), dev(dc.k_raw, "bf16"), dev(dc.v_raw, "bf16"), torch.from_numpy(dc.offsets).cuda()
 
 
-def test_decode_partial_matches_oracle():
+@pytest.mark.parametrize("n_h,n_kv,d", [(16, 2, 128), (32, 1, 64)])
+def test_decode_partial_matches_oracle(n_h, n_kv, d):
     lens = [0, 7, 129, 2000, 64]
-    dc, q, k, v, off = _decode_case(lens, 16, 2, 61)
-    o = torch.empty((len(lens), 16, 128), dtype=torch.float32, device="cuda")
-    lse = torch.empty((len(lens), 16), dtype=torch.float32, device="cuda")
-    ws = torch.zeros(B.cp_workspace_size(B.CP_OP_DECODE, len(lens), 16, 128, 32), dtype=torch.uint8, device="cuda")
-    B.cp_decode_partial(q, k, v, off, 16, 2, 32, 1 / math.sqrt(128), o, lse, ws)
+    dc = synth.make_decode(len(lens), n_h, n_kv, d, lens, 61 + d, 0.5)
+    q, k, v = dev(dc.q_raw, "bf16"), dev(dc.k_raw, "bf16"), dev(dc.v_raw, "bf16")
+    off = torch.from_numpy(dc.offsets).cuda()
+    o = torch.empty((len(lens), n_h, d), dtype=torch.float32, device="cuda")
+    lse = torch.empty((len(lens), n_h), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(B.cp_workspace_size(B.CP_OP_DECODE, len(lens), n_h, d, 32), dtype=torch.uint8, device="cuda")
+    B.cp_decode_partial(q, k, v, off, n_h, n_kv, 32, 1 / math.sqrt(d), o, lse, ws)
     B.cp_check_status(ws)
     o_ref, l_ref = OD.decode(dc.q, dc.k, dc.v, dc.offsets)
     check(o.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "bf16", "decode partial")

@@ -1,8 +1,13 @@
 """GPU parity at the full workload sizes, in the launch configuration the
 bench times, on sampled rows the fp64 reference computes one by one.
 
-Samples always include the first and last row of every chunk (and every
-sequence), plus seeded random rows."""
+Every prefill workload is checked on N_SAMPLE = 2048 query tokens (all heads
+of each), which always include the first and last row of every chunk of the
+load-balanced plan and of every sequence, plus seeded random rows. Besides the
+workload's own inputs, the 128K and varlen workloads also run with Q scaled by
+8 ("peaked": the softmax concentrates on a few keys, so |O| is of order 0.5
+rather than 0.5/sqrt(keys) and the absolute bounds bite). Scaling bf16 values
+by a power of two is exact, so the reference sees the same Q the GPU does."""
 import math
 
 import numpy as np
@@ -15,9 +20,11 @@ from oracle import attention as OA
 from oracle import decode as OD
 from oracle import plan as OP
 
-from gpu_util import check, sample_rows
+from gpu_util import check, oracle_rows, sample_rows
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+N_SAMPLE = 2048
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -28,11 +35,18 @@ def _cuda():
 
 
 def _host_kv(w, n_rows):
+    """K and V as stored (bf16 values), widened to float64 once for the reference."""
     k = synth.stored_values(synth.normal_rows(w["seed"], synth.TENSOR_K, n_rows, (w["n_kv"], w["d"]), w["std"]),
                             "bf16")[0]
     v = synth.stored_values(synth.normal_rows(w["seed"], synth.TENSOR_V, n_rows, (w["n_kv"], w["d"]), w["std"]),
                             "bf16")[0]
-    return k, v
+    return k.astype(np.float64), v.astype(np.float64)
+
+
+def _host_q(w, n_rows, rows, q_mult):
+    qs = synth.stored_values(synth.normal_rows(w["seed"], synth.TENSOR_Q, n_rows, (w["n_h"], w["d"]), w["std"], rows),
+                             "bf16")[0]
+    return qs.astype(np.float64) * q_mult
 
 
 def _dev(w, tid, n_rows, heads):
@@ -49,12 +63,20 @@ def _chunk_edges(lengths, starts, n_ranks):
     return must
 
 
-@pytest.mark.parametrize("merge", ["final", "fused"])
-def test_prefill_128k_pass_kv(merge):
-    """The headline step (separate 8-way merge) and its fused-merge variant."""
+def _gather(out, lse, rows):
+    sel = torch.from_numpy(rows).cuda()
+    return out[sel].float().cpu().numpy(), lse[sel].cpu().numpy()
+
+
+@pytest.mark.parametrize("merge,q_mult", [("final", 1.0), ("fused", 1.0), ("final", 8.0)])
+def test_prefill_128k_pass_kv(merge, q_mult):
+    """The headline step (separate 8-way merge), its fused-merge variant, and
+    the headline step on peaked queries."""
     w = synth.WORKLOADS["prefill_128k"]
     t, n_h, n_kv, d, n = w["t"], w["n_h"], w["n_kv"], w["d"], w["n_ranks"]
     q, k, v = _dev(w, synth.TENSOR_Q, t, n_h), _dev(w, synth.TENSOR_K, t, n_kv), _dev(w, synth.TENSOR_V, t, n_kv)
+    if q_mult != 1.0:
+        q.mul_(q_mult)
     segs = [ring.Segment(t, 0, 0, 0)]
     sched = ring.RingSchedule(segs, segs, n, B.CP_PASS_KV)
     out = torch.empty((t, n_h, d), dtype=torch.bfloat16, device="cuda")
@@ -62,45 +84,51 @@ def test_prefill_128k_pass_kv(merge):
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
     ring.run_ring(sched, q, k, v, n_h, n_kv, out, lse, workspace=ws, merge=merge)
     B.cp_check_status(ws)
-    rows = sample_rows(np.random.default_rng(2), t, 1024, _chunk_edges([t], [0], n))
-    o_gpu = out[torch.from_numpy(rows).cuda()].float().cpu().numpy()
-    l_gpu = lse[torch.from_numpy(rows).cuda()].cpu().numpy()
-    del q, out, lse
+    rows = sample_rows(np.random.default_rng(2 + int(q_mult)), t, N_SAMPLE, _chunk_edges([t], [0], n))
+    assert rows.size >= N_SAMPLE
+    o_gpu, l_gpu = _gather(out, lse, rows)
+    del q, k, v, out, lse
+    torch.cuda.empty_cache()
     kh, vh = _host_kv(w, t)
-    qs = synth.stored_values(synth.normal_rows(w["seed"], synth.TENSOR_Q, t, (n_h, d), w["std"], rows), "bf16")[0]
-    o_ref, l_ref = OA.attention(qs, kh, vh, rows, np.arange(t))
-    check(o_gpu, l_gpu, o_ref, l_ref, "bf16", "prefill_128k")
+    qs = _host_q(w, t, rows, q_mult)
+    o_ref, l_ref = oracle_rows(lambda a, b: OA.attention(qs[a:b], kh, vh, rows[a:b], np.arange(t)), rows.size)
+    check(o_gpu, l_gpu, o_ref, l_ref, "bf16", f"prefill_128k merge={merge} q*{q_mult}")
 
 
-def test_persistent_kv_pass_q_and_pass_kv_agree():
+def test_persistent_kv_pass_q_and_pass_kv():
+    """Both ring variants on the persistent-KV workload: each against the
+    reference on the sampled rows, and the two against each other on every row."""
     w = synth.WORKLOADS["persistent_kv"]
     t, p, n_h, n_kv, d, n = w["t"], w["p"], w["n_h"], w["n_kv"], w["d"], w["n_ranks"]
     q = _dev(w, synth.TENSOR_Q, t, n_h)
     k, v = _dev(w, synth.TENSOR_K, p + t, n_kv), _dev(w, synth.TENSOR_V, p + t, n_kv)
     q_segs = [ring.Segment(t, 0, p, 0)]
     kv_segs = [ring.Segment(p, 0, 0, 0), ring.Segment(t, p, p, 0)]
-    outs = {}
+    # query rows at positions P and P+T-1 and the chunk edges of the new tokens' plan
+    must = [0, t - 1] + _chunk_edges([t], [0], n)
+    rows = sample_rows(np.random.default_rng(3), t, N_SAMPLE, must)
+    assert rows.size >= N_SAMPLE
+    outs, got = {}, {}
     for variant in (B.CP_PASS_Q, B.CP_PASS_KV):
         sched = ring.RingSchedule(q_segs, kv_segs, n, variant)
         out = torch.empty((t, n_h, d), dtype=torch.bfloat16, device="cuda")
         lse = torch.empty((t, n_h), dtype=torch.float32, device="cuda")
-        ring.run_ring(sched, q, k, v, n_h, n_kv, out, lse)
+        ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+        ring.run_ring(sched, q, k, v, n_h, n_kv, out, lse, workspace=ws)
+        B.cp_check_status(ws)
         outs[variant] = (out, lse)
-    torch.cuda.synchronize()
-    # the two ring variants agree on every row
+        got[variant] = _gather(out, lse, rows)
     diff = (outs[B.CP_PASS_Q][0].float() - outs[B.CP_PASS_KV][0].float()).abs().max().item()
     ldiff = (outs[B.CP_PASS_Q][1] - outs[B.CP_PASS_KV][1]).abs().max().item()
     assert diff <= 2e-2 and ldiff <= 1e-3, (diff, ldiff)
-    must = [0, t - 1] + _chunk_edges([t], [0], n)
-    rows = sample_rows(np.random.default_rng(3), t, 64, must)
-    sel = torch.from_numpy(rows).cuda()
-    o_gpu = outs[B.CP_PASS_Q][0][sel].float().cpu().numpy()
-    l_gpu = outs[B.CP_PASS_Q][1][sel].cpu().numpy()
     del outs, q, k, v
+    torch.cuda.empty_cache()
     kh, vh = _host_kv(w, p + t)
-    qs = synth.stored_values(synth.normal_rows(w["seed"], synth.TENSOR_Q, t, (n_h, d), w["std"], rows), "bf16")[0]
-    o_ref, l_ref = OA.attention(qs, kh, vh, p + rows, np.arange(p + t))
-    check(o_gpu, l_gpu, o_ref, l_ref, "bf16", "persistent_kv")
+    qs = _host_q(w, t, rows, 1.0)
+    o_ref, l_ref = oracle_rows(lambda a, b: OA.attention(qs[a:b], kh, vh, p + rows[a:b], np.arange(p + t)),
+                               rows.size, chunk=64)
+    for variant, name in ((B.CP_PASS_Q, "pass-Q"), (B.CP_PASS_KV, "pass-KV")):
+        check(*got[variant], o_ref, l_ref, "bf16", f"persistent_kv {name}")
 
 
 def test_decode_split_full():
@@ -119,16 +147,18 @@ def test_decode_split_full():
     check(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "bf16", "decode_split")
 
 
-@pytest.mark.parametrize("merge", ["fused", "running"])
-def test_varlen_prefill_pass_kv(merge):
+@pytest.mark.parametrize("merge,q_mult", [("fused", 1.0), ("running", 1.0), ("fused", 8.0)])
+def test_varlen_prefill_pass_kv(merge, q_mult):
     """The full varlen workload in both merge modes the bench times (fused is
-    the workload's default)."""
+    the workload's default), and the default on peaked queries."""
     w = synth.WORKLOADS["varlen_prefill"]
     lens = synth.varlen_lengths(w["seed"], w["n_seq"], w["total"])
     total, n_h, n_kv, d, n = w["total"], w["n_h"], w["n_kv"], w["d"], w["n_ranks"]
     starts = np.concatenate([[0], np.cumsum(lens)[:-1]]).astype(np.int64)
     segs = [ring.Segment(int(ln), int(s), 0, i) for i, (ln, s) in enumerate(zip(lens, starts))]
     q = _dev(w, synth.TENSOR_Q, total, n_h)
+    if q_mult != 1.0:
+        q.mul_(q_mult)
     k, v = _dev(w, synth.TENSOR_K, total, n_kv), _dev(w, synth.TENSOR_V, total, n_kv)
     sched = ring.RingSchedule(segs, segs, n, B.CP_PASS_KV)
     out = torch.empty((total, n_h, d), dtype=torch.bfloat16, device="cuda")
@@ -137,22 +167,23 @@ def test_varlen_prefill_pass_kv(merge):
     ring.run_ring(sched, q, k, v, n_h, n_kv, out, lse, workspace=ws, merge=merge)
     B.cp_check_status(ws)
     must = [int(s) for s in starts] + [int(s + ln - 1) for s, ln in zip(starts, lens)]
-    must += _chunk_edges([lens[0]], [0], n)
-    rows = sample_rows(np.random.default_rng(5), total, 128, must)
-    sel = torch.from_numpy(rows).cuda()
-    o_gpu = out[sel].float().cpu().numpy()
-    l_gpu = lse[sel].cpu().numpy()
+    must += _chunk_edges([int(x) for x in lens], [int(s) for s in starts], n)
+    rows = sample_rows(np.random.default_rng(5 + int(q_mult)), total, N_SAMPLE, must)
+    assert rows.size >= N_SAMPLE
+    o_gpu, l_gpu = _gather(out, lse, rows)
     del q, out, lse, k, v
     torch.cuda.empty_cache()
     kh, vh = _host_kv(w, total)
-    qs = synth.stored_values(synth.normal_rows(w["seed"], synth.TENSOR_Q, total, (n_h, d), w["std"], rows), "bf16")[0]
+    qs = _host_q(w, total, rows, q_mult)
     # keys of other sequences are never visible: each sequence is checked against its own keys
     o_ref = np.zeros((rows.size, n_h, d))
     l_ref = np.zeros((rows.size, n_h))
     for s0, ln in zip(starts, lens):
-        sel_rows = np.nonzero((rows >= s0) & (rows < s0 + ln))[0]
-        if sel_rows.size == 0:
+        idx = np.nonzero((rows >= s0) & (rows < s0 + ln))[0]
+        if idx.size == 0:
             continue
-        o_ref[sel_rows], l_ref[sel_rows] = OA.attention(qs[sel_rows], kh[s0:s0 + ln], vh[s0:s0 + ln],
-                                                        rows[sel_rows] - s0, np.arange(ln))
-    check(o_gpu, l_gpu, o_ref, l_ref, "bf16", "varlen_prefill")
+        ks, vs = kh[s0:s0 + ln], vh[s0:s0 + ln]
+        qi, pos = qs[idx], rows[idx] - s0
+        o_ref[idx], l_ref[idx] = oracle_rows(lambda a, b: OA.attention(qi[a:b], ks, vs, pos[a:b], np.arange(ln)),
+                                             idx.size, chunk=64)
+    check(o_gpu, l_gpu, o_ref, l_ref, "bf16", f"varlen_prefill merge={merge} q*{q_mult}")

@@ -47,6 +47,8 @@ def test_shard_plan_bit_exact(lens, n, mode):
     segs = _segs(lens)
     cb, rr, ti = B.cp_shard_plan(_c_segs(segs), len(segs), n, mode)
     ob, orr, oti = OP.shard_plan(segs, n, mode)
+    # the sizes query (NULL arrays) gives the reference plan's array lengths
+    assert B.cp_shard_plan_sizes(_c_segs(segs), len(segs), n, mode) == (sum(len(b) for b in ob), len(orr), len(oti))
     assert np.array_equal(cb, np.array(ob, dtype=np.int64).reshape(len(segs), 2 * n + 1))
     assert list(rr) == orr
     if len(oti) < 2_000_000:
