@@ -368,6 +368,36 @@ def run_ours(args, rank: int, world: int):
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         fused_ms = float(tt.item())
 
+    # the same step with bf16 partial O buffers (cp_attn_partial_bf16_parts, then
+    # cp_attn_merge_bf16_parts): half the partial bytes written and read
+    o_parts16 = o_parts.view(-1).view(torch.bfloat16)[:n_ranks * t * n_h * d].view(n_ranks * t, n_h, d)  # same memory
+
+    def bf16_step():
+        sched = ring.RingSchedule(segs, segs, n_ranks, B.CP_PASS_KV)
+        for s in range(n_ranks):
+            B.cp_attn_partial_bf16_parts(q, k, v, n_h, n_kv, scale, True, sched.ranges, sched.n_ranges,
+                                         sched.step_blocks(s, t), n_ranks, o_parts16, lse_parts, ws)
+        B.cp_attn_merge(o_parts16, lse_parts, n_ranks, t, t, n_h, d, out, lse)
+
+    bf16_ms = None
+    if not args.no_fused:
+        for _ in range(max(2, args.warmup)):
+            bf16_step()
+        barrier()
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            bf16_step()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        B.cp_check_status(ws)
+        bf16_ms = f0.elapsed_time(f1) / args.steps
+    if world > 1 and bf16_ms is not None:
+        tt = torch.tensor([bf16_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        bf16_ms = float(tt.item())
+
     e2e = run_e2e(args, q, k, v, out, lse, o_parts, lse_parts, ws, segs, n_ranks, n_h, n_kv, world, dev,
                   step_flops, barrier) if not args.no_e2e else None
     decode = run_decode(args, dev) if not args.no_decode else None
@@ -404,6 +434,10 @@ def run_ours(args, rank: int, world: int):
             "value": world * step_flops / (fused_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": fused_ms,
             "note": "same step, LSE merge in the partial kernel's epilogue (cp_attn_partial_fused): "
                     "8 launches, one running buffer, no merge pass"},
+        "bf16_partials": None if bf16_ms is None else {
+            "value": world * step_flops / (bf16_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": bf16_ms,
+            "note": "same step with bf16 partial O buffers (cp_attn_partial_bf16_parts + cp_attn_merge_bf16_parts): "
+                    "8 launches + one 8-way merge reading half the partial bytes"},
         "e2e": e2e,
         "gpu_launches": args.steps * (n_ranks + 1),
         "clocks": clk,

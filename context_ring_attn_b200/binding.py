@@ -44,7 +44,7 @@ EXPORTED = (
     "cp_classify_pair", "cp_block_pairs", "cp_ring_comm_volume", "cp_workspace_size",
     "cp_reset_status", "cp_check_status", "cp_attn_partial", "cp_attn_merge", "cp_decode",
     "cp_decode_static", "cp_decode_partial", "cp_select_ring_variant", "cp_attn_partial_fused",
-    "cp_wait_selftest", "cp_decode_static_status",
+    "cp_wait_selftest", "cp_decode_static_status", "cp_attn_partial_bf16_parts", "cp_attn_merge_bf16_parts",
 )
 
 
@@ -101,6 +101,9 @@ def lib() -> ctypes.CDLL:
         "cp_attn_partial_fused": (i32, [vp, vp, vp, i32, i64, i64, i32, i32, i32, f32, i32, P(cp_range), i32,
                                         P(cp_block), i32, vp, vp, i64, i32, vp, vp, sz, vp]),
         "cp_attn_merge": (i32, [vp, vp, i32, i64, i64, i32, i32, vp, i32, vp, vp]),
+        "cp_attn_merge_bf16_parts": (i32, [vp, vp, i32, i64, i64, i32, i32, vp, i32, vp, vp]),
+        "cp_attn_partial_bf16_parts": (i32, [vp, vp, vp, i32, i64, i64, i32, i32, i32, f32, i32, P(cp_range), i32,
+                                             P(cp_block), i32, vp, vp, i64, vp, sz, vp]),
         "cp_decode": (i32, [vp, vp, vp, i32, vp, i32, i64, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]),
         "cp_decode_static": (i32, [vp, vp, vp, i32, vp, i32, i64, i32, i32, i32, i32, f32, vp, vp, vp]),
         "cp_decode_static_status": (i32, [vp]),
@@ -279,9 +282,23 @@ def cp_attn_partial_fused(q, k, v, n_h: int, n_kv: int, softmax_scale: float, ca
 
 def cp_attn_merge(o_parts, lse_parts, n_parts: int, part_stride_rows: int, rows: int, n_h: int, d: int, out,
                   lse_out=None, stream=None) -> None:
-    code = lib().cp_attn_merge(_ptr(o_parts), _ptr(lse_parts), n_parts, part_stride_rows, rows, n_h, d,
-                               _ptr(out), _dtype_code(out), _ptr(lse_out), _stream(stream))
-    _check("cp_attn_merge", code)
+    """LSE merge; o_parts fp32 (cp_attn_merge) or bf16 (cp_attn_merge_bf16_parts), chosen by its dtype."""
+    fn = "cp_attn_merge_bf16_parts" if _dtype_code(o_parts) == CP_BF16 else "cp_attn_merge"
+    code = getattr(lib(), fn)(_ptr(o_parts), _ptr(lse_parts), n_parts, part_stride_rows, rows, n_h, d,
+                              _ptr(out), _dtype_code(out), _ptr(lse_out), _stream(stream))
+    _check(fn, code)
+
+
+def cp_attn_partial_bf16_parts(q, k, v, n_h: int, n_kv: int, softmax_scale: float, causal: bool, ranges,
+                               n_ranges: int, blocks, n_blocks: int, o_part, lse_part, workspace, stream=None) -> None:
+    """cp_attn_partial writing bf16 O partials (o_part bf16 [out_rows, n_h, d]); LSE fp32."""
+    d = int(q.shape[-1])
+    code = lib().cp_attn_partial_bf16_parts(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), int(q.shape[0]),
+                                            int(k.shape[0]), n_h, n_kv, d, float(softmax_scale), int(causal), ranges,
+                                            n_ranges, blocks, n_blocks, _ptr(o_part), _ptr(lse_part),
+                                            int(o_part.shape[0]), _ptr(workspace),
+                                            int(workspace.numel() * workspace.element_size()), _stream(stream))
+    _check("cp_attn_partial_bf16_parts", code)
 
 
 def cp_decode(q, k, v, kv_offsets, n_h: int, n_kv: int, n_splits: int, softmax_scale: float, out, lse_out,

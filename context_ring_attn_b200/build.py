@@ -2,7 +2,6 @@
 
     python -m context_ring_attn_b200.build          # build if sources are newer
     python -m context_ring_attn_b200.build --force  # always rebuild
-    CPK_PAIR_KERNEL=1 python -m context_ring_attn_b200.build --force   # bf16 partial on SM pairs
 """
 from __future__ import annotations
 
@@ -17,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libcpattn.so")
 SOURCES = ["plan.cpp", "capi.cu"]
-HEADERS = ["common.cuh", "work.cuh", "partial_tc.cuh", "partial_tc2.cuh", "partial_simt.cuh", "merge.cuh", "decode.cuh", "exp2_poly.cuh"]
+HEADERS = ["common.cuh", "work.cuh", "partial_tc.cuh", "partial_simt.cuh", "merge.cuh", "decode.cuh", "exp2_poly.cuh"]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
@@ -44,8 +43,6 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     if not force and not _stale():
         return LIB
     tmp = LIB + ".tmp"
-    if os.environ.get("CPK_PAIR_KERNEL") == "1":   # bf16 partial attention on SM pairs
-        extra_flags = (*extra_flags, "-DCPK_PAIR_KERNEL=1")
     cmd = [nvcc_path(), *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC, "-o", tmp,
            *[os.path.join(CSRC, f) for f in SOURCES]]
     if verbose:

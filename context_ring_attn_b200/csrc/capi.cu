@@ -14,7 +14,6 @@
 #include "merge.cuh"
 #include "partial_simt.cuh"
 #include "partial_tc.cuh"
-#include "partial_tc2.cuh"
 #include "work.cuh"
 
 namespace {
@@ -160,32 +159,35 @@ bool build_tables(const cp_range* ranges, const cp_block* blocks, int32_t n_bloc
   return true;
 }
 
-// Tensor maps: Q as [rows][N_KV][G][D] (box 64 x G x 1 x 128/G), K and V as
-// [rows][N_KV][D] (box 64 x 1 x 128), bf16, 128-byte swizzle.
-// Q box: 128 packed rows (128/G tokens x G heads) x 64 columns; K box: k_box_rows keys x 64 columns; V box:
-// 128 keys x 64 columns; 128-byte swizzle.
+// Tensor maps (bf16, 128-byte swizzle): Q as [rows][N_KV][G][HD] with a box of
+// 64 columns x G heads x 1 KV head x 128/G tokens (128 packed query rows);
+// K and V as [rows][N_KV][HD] with a box of 64 columns x 1 KV head x
+// kv_box_rows keys.
 bool make_qkv_maps(CUtensorMap* tm_q, CUtensorMap* tm_k, CUtensorMap* tm_v, const void* q, const void* k,
-                   const void* v, int64_t q_rows, int64_t kv_rows, int n_h, int n_kv, int group, int k_box_rows) {
+                   const void* v, int64_t q_rows, int64_t kv_rows, int n_h, int n_kv, int group, int hd,
+                   int kv_box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint32_t estr4[4] = {1, 1, 1, 1};
+  const cuuint64_t row_bytes = static_cast<cuuint64_t>(hd) * 2;
   {
-    const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(group), static_cast<cuuint64_t>(n_kv),
-                                static_cast<cuuint64_t>(q_rows)};
-    const cuuint64_t strides[3] = {128 * 2, static_cast<cuuint64_t>(group) * 256,
-                                   static_cast<cuuint64_t>(n_h) * 256};
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(hd), static_cast<cuuint64_t>(group),
+                                static_cast<cuuint64_t>(n_kv), static_cast<cuuint64_t>(q_rows)};
+    const cuuint64_t strides[3] = {row_bytes, static_cast<cuuint64_t>(group) * row_bytes,
+                                   static_cast<cuuint64_t>(n_h) * row_bytes};
     const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(group), 1, static_cast<cuuint32_t>(128 / group)};
     if (enc(tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(q), dims, strides, box, estr4,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return false;
   }
-  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(n_kv), static_cast<cuuint64_t>(kv_rows)};
-  const cuuint64_t strides[2] = {128 * 2, static_cast<cuuint64_t>(n_kv) * 256};
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(hd), static_cast<cuuint64_t>(n_kv),
+                              static_cast<cuuint64_t>(kv_rows)};
+  const cuuint64_t strides[2] = {row_bytes, static_cast<cuuint64_t>(n_kv) * row_bytes};
   const void* src[2] = {k, v};
   CUtensorMap* dst[2] = {tm_k, tm_v};
   for (int i = 0; i < 2; ++i) {
-    const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(i == 0 ? k_box_rows : 128)};
+    const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kv_box_rows)};
     if (enc(dst[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(src[i]), dims, strides, box, estr4,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -195,13 +197,6 @@ bool make_qkv_maps(CUtensorMap* tm_q, CUtensorMap* tm_k, CUtensorMap* tm_v, cons
 }
 
 constexpr size_t kStatusBytes = 256;
-
-#ifndef CPK_PAIR_KERNEL
-#define CPK_PAIR_KERNEL 0
-#endif
-// bf16 partial attention on single SMs (default) or on SM pairs (cta_group::2,
-// built with -DCPK_PAIR_KERNEL=1: parity-tested, slower so far)
-constexpr bool kPairKernel = CPK_PAIR_KERNEL != 0;
 
 inline size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -338,6 +333,22 @@ cp_status decode_launch(const DecodeShape& s, const void* q, const void* k, cons
                               lse_out, ws, stream);
 }
 
+// One launch of the tensor-core partial kernel per work table.
+template <int HD>
+cp_status launch_partial_tc(tc::Params& params, const std::vector<WorkTable>& tables, int n_kv, cudaStream_t stream) {
+  if (cudaFuncSetAttribute(tc::partial_bf16_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           tc::Cfg<HD>::kSmemBytes) != cudaSuccess)
+    return CP_ERR_CUDA;
+  for (const WorkTable& wt : tables) {
+    if (wt.total_tiles == 0) continue;
+    std::memcpy(&params.wt, &wt, sizeof(WorkTable));
+    dim3 grid(wt.total_tiles, n_kv);
+    tc::partial_bf16_kernel<HD><<<grid, tc::kThreads, tc::Cfg<HD>::kSmemBytes, stream>>>(params);
+    if (last_cuda_status() != CP_OK) return CP_ERR_CUDA;
+  }
+  return CP_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -397,8 +408,8 @@ static cp_status partial_impl(const void* q, const void* k, const void* v, cp_dt
                               int32_t causal, const cp_range* ranges, int32_t n_ranges, const cp_block* blocks,
                               int32_t n_blocks, float* o_part, float* lse_part, int64_t out_rows, int32_t accumulate,
                               void* out_final, void* workspace, size_t ws_bytes, void* cuda_stream) {
-  // ---- arguments
-  if (!q || !k || !v || !o_part || !lse_part) return CP_ERR_INVALID_ARG;
+  // ---- arguments (o_part is not read or written when every row goes to out_final unmerged)
+  if (!q || !k || !v || !lse_part || (!o_part && (accumulate || !out_final))) return CP_ERR_INVALID_ARG;
   const bool fused = accumulate != 0 || out_final != nullptr;
   if (fused && dtype != CP_BF16) return CP_ERR_UNSUPPORTED;
   if (out_final && !aligned(out_final, 16)) return CP_ERR_INVALID_ARG;
@@ -409,7 +420,7 @@ static cp_status partial_impl(const void* q, const void* k, const void* v, cp_dt
   if (!workspace || ws_bytes < kStatusBytes || !aligned(workspace, 256)) return CP_ERR_WORKSPACE;
   const int group = n_h / n_kv;
   if (dtype == CP_BF16) {
-    if (d != 128 || ilog2_exact(group) < 0 || group > 128) return CP_ERR_UNSUPPORTED;
+    if ((d != 64 && d != 128) || ilog2_exact(group) < 0 || group > 128) return CP_ERR_UNSUPPORTED;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return CP_ERR_INVALID_ARG;
     if (q_rows >= (int64_t(1) << 31) || kv_rows >= (int64_t(1) << 31)) return CP_ERR_UNSUPPORTED;
   } else if (dtype == CP_F32) {
@@ -418,7 +429,7 @@ static cp_status partial_impl(const void* q, const void* k, const void* v, cp_dt
   } else {
     return CP_ERR_UNSUPPORTED;
   }
-  if (!aligned(o_part, 16) || !aligned(lse_part, 4)) return CP_ERR_INVALID_ARG;
+  if ((o_part && !aligned(o_part, 16)) || !aligned(lse_part, 4)) return CP_ERR_INVALID_ARG;
   for (int32_t b = 0; b < n_blocks; ++b) {
     const cp_block& bl = blocks[b];
     if (bl.q_begin < 0 || bl.q_count < 0 || bl.kv_begin < 0 || bl.kv_count < 0) return CP_ERR_INVALID_ARG;
@@ -459,36 +470,12 @@ static cp_status partial_impl(const void* q, const void* k, const void* v, cp_dt
   uint32_t* status = static_cast<uint32_t*>(workspace);
   const float log2e = 1.4426950408889634f;
 
-  if (dtype == CP_BF16 && kPairKernel) {
-    static tc2::Params params;  // large: kept off the stack; copied at launch
-    static std::mutex mu;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!make_qkv_maps(&params.tm_q, &params.tm_k, &params.tm_v, q, k, v, q_rows, kv_rows, n_h, n_kv, group, 64))
-      return CP_ERR_CUDA;
-    params.o_part = o_part;
-    params.lse_part = lse_part;
-    params.out_final = static_cast<__nv_bfloat16*>(out_final);
-    params.accumulate = accumulate != 0;
-    params.status = status;
-    params.n_h = n_h;
-    params.log2_group = ilog2_exact(group);
-    params.causal = causal != 0;
-    params.scale_log2 = softmax_scale * log2e;
-    if (cudaFuncSetAttribute(tc2::partial_bf16_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             tc2::kSmemBytes) != cudaSuccess)
-      return CP_ERR_CUDA;
-    for (const WorkTable& wt : tables) {
-      if (wt.total_tiles == 0) continue;
-      std::memcpy(&params.wt, &wt, sizeof(WorkTable));
-      dim3 grid(2 * wt.total_tiles, n_kv);   // one cluster of two CTAs per 256-row tile
-      tc2::partial_bf16_pair_kernel<<<grid, tc2::kThreads, tc2::kSmemBytes, stream>>>(params);
-      if (last_cuda_status() != CP_OK) return CP_ERR_CUDA;
-    }
-  } else if (dtype == CP_BF16) {
+  if (dtype == CP_BF16) {
     static tc::Params params;  // large: kept off the stack; copied at launch
     static std::mutex mu;
     std::lock_guard<std::mutex> lock(mu);
-    if (!make_qkv_maps(&params.tm_q, &params.tm_k, &params.tm_v, q, k, v, q_rows, kv_rows, n_h, n_kv, group, 128))
+    if (!make_qkv_maps(&params.tm_q, &params.tm_k, &params.tm_v, q, k, v, q_rows, kv_rows, n_h, n_kv, group, d,
+                       tc::BN))
       return CP_ERR_CUDA;
     params.o_part = o_part;
     params.lse_part = lse_part;
@@ -499,16 +486,9 @@ static cp_status partial_impl(const void* q, const void* k, const void* v, cp_dt
     params.log2_group = ilog2_exact(group);
     params.causal = causal != 0;
     params.scale_log2 = softmax_scale * log2e;
-    if (cudaFuncSetAttribute(tc::partial_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             tc::kSmemBytes) != cudaSuccess)
-      return CP_ERR_CUDA;
-    for (const WorkTable& wt : tables) {
-      if (wt.total_tiles == 0) continue;
-      std::memcpy(&params.wt, &wt, sizeof(WorkTable));
-      dim3 grid(wt.total_tiles, n_kv);
-      tc::partial_bf16_kernel<<<grid, tc::kThreads, tc::kSmemBytes, stream>>>(params);
-      if (last_cuda_status() != CP_OK) return CP_ERR_CUDA;
-    }
+    const cp_status st = d == 64 ? launch_partial_tc<64>(params, tables, n_kv, stream)
+                                 : launch_partial_tc<128>(params, tables, n_kv, stream);
+    if (st != CP_OK) return st;
   } else {
     static simt::Params params;
     static std::mutex mu;
@@ -556,13 +536,23 @@ cp_status cp_attn_partial_fused(const void* q, const void* k, const void* v, cp_
                       n_blocks, o_acc, lse_acc, out_rows, accumulate, out, workspace, ws_bytes, cuda_stream);
 }
 
-cp_status cp_attn_merge(const float* o_parts, const float* lse_parts, int32_t n_parts, int64_t part_stride_rows,
-                        int64_t rows, int32_t n_h, int32_t d, void* out, cp_dtype out_dtype, float* lse_out,
-                        void* cuda_stream) {
+cp_status cp_attn_partial_bf16_parts(const void* q, const void* k, const void* v, cp_dtype dtype, int64_t q_rows,
+                                     int64_t kv_rows, int32_t n_h, int32_t n_kv, int32_t d, float softmax_scale,
+                                     int32_t causal, const cp_range* ranges, int32_t n_ranges, const cp_block* blocks,
+                                     int32_t n_blocks, void* o_part, float* lse_part, int64_t out_rows, void* workspace,
+                                     size_t ws_bytes, void* cuda_stream) {
+  if (!o_part) return CP_ERR_INVALID_ARG;
+  return partial_impl(q, k, v, dtype, q_rows, kv_rows, n_h, n_kv, d, softmax_scale, causal, ranges, n_ranges, blocks,
+                      n_blocks, nullptr, lse_part, out_rows, 0, o_part, workspace, ws_bytes, cuda_stream);
+}
+
+static cp_status merge_impl(const void* o_parts, cp_dtype parts_dtype, const float* lse_parts, int32_t n_parts,
+                            int64_t part_stride_rows, int64_t rows, int32_t n_h, int32_t d, void* out,
+                            cp_dtype out_dtype, float* lse_out, void* cuda_stream) {
   if (!o_parts || !lse_parts || !out) return CP_ERR_INVALID_ARG;
   if (n_parts < 1 || rows < 0 || n_h < 1 || d < 4 || (d & 3)) return CP_ERR_INVALID_ARG;
   if (n_parts > 1 && part_stride_rows < rows) return CP_ERR_INVALID_ARG;
-  if (!aligned(o_parts, 16) || !aligned(lse_parts, 4)) return CP_ERR_INVALID_ARG;
+  if (!aligned(o_parts, parts_dtype == CP_F32 ? 16 : 8) || !aligned(lse_parts, 4)) return CP_ERR_INVALID_ARG;
   if (out_dtype == CP_F32) {
     if (!aligned(out, 16)) return CP_ERR_INVALID_ARG;
   } else if (out_dtype == CP_BF16) {
@@ -575,7 +565,7 @@ cp_status cp_attn_merge(const float* o_parts, const float* lse_parts, int32_t n_
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   const int64_t o_stride = part_stride_rows * n_h * d;
   const int64_t l_stride = part_stride_rows * n_h;
-  // (row, head) pairs per warp and round: 8 float4 loads per lane split over the parts
+  // (row, head) pairs per warp and round: 8 four-element loads per lane split over the parts
   const int c = n_parts > 4 ? 8 : n_parts > 2 ? 4 : 2;
   const int r = 8 / c;
   const int64_t warps_per_block = merge::kThreads / 32;
@@ -583,20 +573,41 @@ cp_status cp_attn_merge(const float* o_parts, const float* lse_parts, int32_t n_
   grid = std::min<int64_t>(grid, 148 * 32);
   const unsigned g = static_cast<unsigned>(grid);
   const unsigned t = merge::kThreads;
-#define CP_MERGE_LAUNCH(OutT, R_)                                                                          \
-  merge::merge_kernel<OutT, R_><<<g, t, 0, stream>>>(o_parts, lse_parts, n_parts, o_stride, l_stride, n_rowheads, d, \
-                                                     static_cast<OutT*>(out), lse_out)
-  if (out_dtype == CP_F32) {
-    if (r == 1) CP_MERGE_LAUNCH(float, 1);
-    else if (r == 2) CP_MERGE_LAUNCH(float, 2);
-    else CP_MERGE_LAUNCH(float, 4);
+#define CP_MERGE_LAUNCH(InT, OutT, R_)                                                                         \
+  merge::merge_kernel<InT, OutT, R_><<<g, t, 0, stream>>>(static_cast<const InT*>(o_parts), lse_parts, n_parts,  \
+                                                          o_stride, l_stride, n_rowheads, d, static_cast<OutT*>(out), \
+                                                          lse_out)
+#define CP_MERGE_BY_R(InT, OutT)                \
+  do {                                          \
+    if (r == 1) CP_MERGE_LAUNCH(InT, OutT, 1);  \
+    else if (r == 2) CP_MERGE_LAUNCH(InT, OutT, 2); \
+    else CP_MERGE_LAUNCH(InT, OutT, 4);         \
+  } while (0)
+  if (parts_dtype == CP_F32) {
+    if (out_dtype == CP_F32) CP_MERGE_BY_R(float, float);
+    else CP_MERGE_BY_R(float, __nv_bfloat16);
   } else {
-    if (r == 1) CP_MERGE_LAUNCH(__nv_bfloat16, 1);
-    else if (r == 2) CP_MERGE_LAUNCH(__nv_bfloat16, 2);
-    else CP_MERGE_LAUNCH(__nv_bfloat16, 4);
+    if (out_dtype == CP_F32) CP_MERGE_BY_R(__nv_bfloat16, float);
+    else CP_MERGE_BY_R(__nv_bfloat16, __nv_bfloat16);
   }
+#undef CP_MERGE_BY_R
 #undef CP_MERGE_LAUNCH
   return last_cuda_status();
+}
+
+cp_status cp_attn_merge(const float* o_parts, const float* lse_parts, int32_t n_parts, int64_t part_stride_rows,
+                        int64_t rows, int32_t n_h, int32_t d, void* out, cp_dtype out_dtype, float* lse_out,
+                        void* cuda_stream) {
+  return merge_impl(o_parts, CP_F32, lse_parts, n_parts, part_stride_rows, rows, n_h, d, out, out_dtype, lse_out,
+                    cuda_stream);
+}
+
+cp_status cp_attn_merge_bf16_parts(const void* o_parts, const float* lse_parts, int32_t n_parts,
+                                   int64_t part_stride_rows, int64_t rows, int32_t n_h, int32_t d, void* out,
+                                   cp_dtype out_dtype, float* lse_out, void* cuda_stream) {
+  if (out == o_parts && out_dtype == CP_F32) return CP_ERR_INVALID_ARG;   // in place needs matching element sizes
+  return merge_impl(o_parts, CP_BF16, lse_parts, n_parts, part_stride_rows, rows, n_h, d, out, out_dtype, lse_out,
+                    cuda_stream);
 }
 
 static cp_status decode_impl(const void* q, const void* k, const void* v, cp_dtype dtype, const int64_t* kv_offsets,

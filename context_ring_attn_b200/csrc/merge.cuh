@@ -26,6 +26,16 @@ namespace merge {
 constexpr int kThreads = 256;
 constexpr int kLoads = 8;   // float4 loads per lane per round
 
+// Four consecutive partial elements (fp32, or bf16 partial buffers) as fp32,
+// streamed (read once).
+__device__ __forceinline__ float4 load4(const float* src) { return __ldcs(reinterpret_cast<const float4*>(src)); }
+
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* src) {
+  const uint2 u = __ldcs(reinterpret_cast<const uint2*>(src));
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u), __uint_as_float(u.y << 16),
+                     __uint_as_float(u.y & 0xffff0000u));
+}
+
 __device__ __forceinline__ void store4(float* dst, float4 v) { *reinterpret_cast<float4*>(dst) = v; }
 
 __device__ __forceinline__ void store4(__nv_bfloat16* dst, float4 v) {
@@ -36,8 +46,9 @@ __device__ __forceinline__ void store4(__nv_bfloat16* dst, float4 v) {
 }
 
 // o_parts / lse_parts carry no __restrict__: out and lse_out may alias part 0.
-template <typename OutT, int R>
-__global__ void __launch_bounds__(kThreads, R <= 2 ? 3 : 2) merge_kernel(const float* o_parts,
+// InT: fp32 partials, or bf16 partial buffers (rounded O, fp32 LSE).
+template <typename InT, typename OutT, int R>
+__global__ void __launch_bounds__(kThreads, R <= 2 ? 3 : 2) merge_kernel(const InT* o_parts,
                                                           const float* lse_parts, int n_parts,
                                                           int64_t o_stride, int64_t l_stride, int64_t n_rowheads,
                                                           int d, OutT* out, float* lse_out) {
@@ -73,7 +84,7 @@ __global__ void __launch_bounds__(kThreads, R <= 2 ? 3 : 2) merge_kernel(const f
             x[r][c] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (rh < n_rowheads && j < n_parts) {
               lj[r][c] = lse_parts[j * l_stride + rh];
-              if (active) x[r][c] = __ldcs(reinterpret_cast<const float4*>(o_parts + j * o_stride + rh * d) + vi);
+              if (active) x[r][c] = load4(o_parts + j * o_stride + rh * d + vi * 4);
             }
           }
         }

@@ -30,6 +30,8 @@
 //              overlaps the other tile's MMAs (ping-pong).
 // Two threads per row halve the latency of a softmax step, which otherwise
 // exceeds the MMA time of one tile and stalls the ping-pong.
+// Head dims 64 and 128 are two instantiations (a row is HD/64 swizzle columns
+// of 64 bf16; S = Q K^T takes HD/16 MMA steps and O has HD columns).
 // TMEM (512 columns): S_a 0, S_b 128, O_a 256, O_b 384. Each half row's P
 // (bf16 pairs) goes over the first 32 of its own 64 S columns. tcgen05 operations of one thread complete in issue order, so the
 // completion of S_x(j+1) also means O_x += P_x(j) V_j has completed.
@@ -43,51 +45,58 @@ namespace tc {
 
 constexpr int BM = 128;                      // packed query rows per tile
 constexpr int BN = 128;                      // keys per KV tile
-constexpr int HD = 128;                      // head dim
 constexpr int kQTiles = 2;                   // query tiles per CTA
 constexpr int kHalfBytes = 128 * 128;        // 128 rows x 64 bf16 (one 128-byte swizzle column)
-constexpr int kTileBytes = 2 * kHalfBytes;   // 128 rows x 128 bf16
-constexpr int kKStages = 3;
-constexpr int kVStages = 2;
 constexpr int kSoftmaxWarps = 16;
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
 constexpr int kThreads = 576;
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQTiles * kTileBytes;
-constexpr int kOffV = kOffK + kKStages * kTileBytes;
-constexpr int kOffBar = kOffV + kVStages * kTileBytes;
 constexpr int kNumBars = 24;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kOffXch = kOffMisc + 16;                 // [tile][half][row] f32: half-row max, then sum
-constexpr int kSmemNeeded = kOffXch + kQTiles * 2 * BM * 4;
 constexpr int kSmemMax = 232448;                     // 227 KB per block on sm_100
-// The dynamic shared window starts 1024-aligned in practice; whatever slack is
-// left covers a smaller alignment, and the kernel checks it at run time.
-constexpr int kSmemBytes = kSmemNeeded + 1024 <= kSmemMax ? kSmemNeeded + 1024 : kSmemMax;
-static_assert(kSmemNeeded <= kSmemMax, "shared memory plan exceeds 227 KB");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;     // + tile * 128
-constexpr uint32_t kColO = 256;   // + tile * 128
+constexpr uint32_t kColO = 256;   // + tile * 128 (HD columns used)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled when the max grows by > 2^8
 constexpr int kPolyPairsPer8 = 1;          // of every 8 column pairs, this many take the polynomial exp2
+
+// Shared-memory plan of a head dim HD (64 or 128): a Q, K or V tile of 128
+// rows is HD/64 swizzle columns of 16 KB each.
+template <int HD>
+struct Cfg {
+  static constexpr int kHalves = HD / 64;
+  static constexpr int kTileBytes = kHalves * kHalfBytes;   // 128 rows x HD bf16
+  static constexpr int kKStages = 3;
+  static constexpr int kVStages = HD == 128 ? 2 : 3;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQTiles * kTileBytes;
+  static constexpr int kOffV = kOffK + kKStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kOffXch = kOffMisc + 16;           // [tile][half][row] f32: half-row max, then sum
+  static constexpr int kSmemNeeded = kOffXch + kQTiles * 2 * BM * 4;
+  // The dynamic shared window starts 1024-aligned in practice; whatever slack is
+  // left covers a smaller alignment, and the kernel checks it at run time.
+  static constexpr int kSmemBytes = kSmemNeeded + 1024 <= kSmemMax ? kSmemNeeded + 1024 : kSmemMax;
+  static_assert(kSmemNeeded <= kSmemMax, "shared memory plan exceeds 227 KB");
+  static_assert(kKStages <= 3 && kVStages <= 3, "barrier slots hold at most 3 stages");
+};
 
 // barrier slots
 enum {
   B_Q_FULL = 0,
   B_K_FULL = 1,     // +stage (3)
   B_K_EMPTY = 4,    // +stage (3)
-  B_V_FULL = 7,     // +stage (2)
-  B_V_EMPTY = 9,    // +stage (2)
-  B_S_FULL = 11,    // +tile: S_x(j) is in TMEM (and O_x += P_x(j-1) V is done)
-  B_P_FULL = 13,    // +tile (8 arrivals): P_x(j) is in TMEM
-  B_O_DONE = 15,    // +tile: O_x += P_x(j) V_j has completed
-  B_DRAIN = 17
+  B_V_FULL = 7,     // +stage (3)
+  B_V_EMPTY = 10,   // +stage (3)
+  B_S_FULL = 13,    // +tile: S_x(j) is in TMEM (and O_x += P_x(j-1) V is done)
+  B_P_FULL = 15,    // +tile (8 arrivals): P_x(j) is in TMEM
+  B_O_DONE = 17,    // +tile: O_x += P_x(j) V_j has completed
+  B_DRAIN = 19
 };
 
 struct Params {
-  CUtensorMap tm_q;  // [q_rows][N_KV][G][128] bf16, box {64, G, 1, 128/G}
-  CUtensorMap tm_k;  // [kv_rows][N_KV][128] bf16, box {64, 1, 128}
+  CUtensorMap tm_q;  // [q_rows][N_KV][G][HD] bf16, box {64, G, 1, 128/G}
+  CUtensorMap tm_k;  // [kv_rows][N_KV][HD] bf16, box {64, 1, 128}
   CUtensorMap tm_v;
   float* o_part;
   float* lse_part;
@@ -188,7 +197,15 @@ __device__ __forceinline__ float half_row_exps(uint32_t s_col, float sl2, float 
 
 // 18 warps put five on two of the four schedulers, whose register files hold
 // 16K registers each: at most 102 per thread, so 96.
+template <int HD>
 __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Params p) {
+  using C = Cfg<HD>;
+  constexpr int kTileBytes = C::kTileBytes;
+  constexpr int kKStages = C::kKStages;
+  constexpr int kVStages = C::kVStages;
+  constexpr int kOffQ = C::kOffQ, kOffK = C::kOffK, kOffV = C::kOffV, kOffBar = C::kOffBar;
+  constexpr int kOffMisc = C::kOffMisc, kOffXch = C::kOffXch;
+  constexpr int kSmemNeeded = C::kSmemNeeded, kSmemBytes = C::kSmemBytes;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
@@ -257,13 +274,14 @@ __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Para
       const CUtensorMap* map = is_k ? &p.tm_k : &p.tm_v;
       uint64_t* full = &bars[is_k ? B_K_FULL : B_V_FULL];
       uint64_t* empty = &bars[is_k ? B_K_EMPTY : B_V_EMPTY];
-      uint32_t issued[kKStages] = {0u, 0u, 0u};
+      uint32_t issued[3] = {0u, 0u, 0u};
       if (is_k) {
         mbar_arrive_expect_tx(&bars[B_Q_FULL], kQTiles * kTileBytes);
         for (int t = 0; t < kQTiles; ++t) {
           const int row = static_cast<int>(q_row0) + t * tok_per_tile;
-          tma_load_4d(sQ + t * kTileBytes, &p.tm_q, &bars[B_Q_FULL], 0, 0, kvh, row);
-          tma_load_4d(sQ + t * kTileBytes + kHalfBytes, &p.tm_q, &bars[B_Q_FULL], 64, 0, kvh, row);
+#pragma unroll
+          for (int h = 0; h < C::kHalves; ++h)
+            tma_load_4d(sQ + t * kTileBytes + h * kHalfBytes, &p.tm_q, &bars[B_Q_FULL], h * 64, 0, kvh, row);
         }
       }
       int it = 0;
@@ -278,8 +296,9 @@ __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Para
           const int key_row = static_cast<int>(kr.row0 + k0);
           if (it >= n_st && !mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[st], kTileBytes);
-          tma_load_3d(base + st * kTileBytes, map, &full[st], 0, kvh, key_row);
-          tma_load_3d(base + st * kTileBytes + kHalfBytes, map, &full[st], 64, kvh, key_row);
+#pragma unroll
+          for (int h = 0; h < C::kHalves; ++h)
+            tma_load_3d(base + st * kTileBytes + h * kHalfBytes, map, &full[st], h * 64, kvh, key_row);
           issued[st] += 1;
         }
       }
@@ -315,7 +334,7 @@ __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Para
         for (int kk = 0; kk < BN / 16; ++kk) {
           // keys 16kk..16kk+15 as bf16 pairs: the P of each half sits in its own first 32 S columns
           const uint32_t p_addr = tmem + kColS + x * BN + (kk >> 2) * 64 + (kk & 3) * 8;
-          umma_bf16_ts(tmem + kColO + x * HD, p_addr, vd + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o,
+          umma_bf16_ts(tmem + kColO + x * 128, p_addr, vd + static_cast<uint64_t>((kk * 2048) >> 4), idesc_o,
                        (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&bars[B_O_DONE + x]);
@@ -355,7 +374,7 @@ __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Para
     const int row = quarter * 32 + lane;    // packed row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_col = tmem + lane_base + kColS + x * BN + hf * 64;   // this thread's S columns
-    const uint32_t o_col = tmem + lane_base + kColO + x * HD + hf * 64;   // its O columns
+    const uint32_t o_col = tmem + lane_base + kColO + x * 128 + hf * (HD / 2);   // its O columns
     float* xch_mine = reinterpret_cast<float*>(smem + kOffXch) + (x * 2 + hf) * BM + row;
     const float* xch_peer = reinterpret_cast<const float*>(smem + kOffXch) + (x * 2 + (hf ^ 1)) * BM + row;
     const uint32_t pair_bar = 1 + x * 4 + quarter;   // named barrier of the two warps sharing these rows
@@ -457,7 +476,7 @@ __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Para
         // O_x holds every earlier PV (see S_FULL above): rescale this half in place if needed
         if (it > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < HD / 32; ++c) {
             uint32_t o[16];
             tmem_ld16(o_col + c * 16, o);
             tmem_ld_wait();
@@ -506,11 +525,11 @@ __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Para
         lse_new = mx + logf(sum);
       }
     }
-    float* dst = p.o_part + out_idx * HD + hf * 64;
+    float* dst = p.o_part + out_idx * HD + hf * (HD / 2);
     if (done_ok) {
       if (n_iter > 0) tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < HD / 64; ++c) {
         uint32_t o[32];
         if (n_iter > 0) {
           tmem_ld32(o_col + c * 32, o);
@@ -534,7 +553,7 @@ __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Para
             }
           }
           if (p.out_final) {
-            uint4* fo = reinterpret_cast<uint4*>(p.out_final + out_idx * HD + hf * 64 + c * 32);
+            uint4* fo = reinterpret_cast<uint4*>(p.out_final + out_idx * HD + hf * (HD / 2) + c * 32);
 #pragma unroll
             for (int i = 0; i < 32; i += 8)
               fo[i >> 3] = make_uint4(pack_bf16x2(r[i], r[i + 1]), pack_bf16x2(r[i + 2], r[i + 3]),

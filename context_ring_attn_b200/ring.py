@@ -65,8 +65,8 @@ def _nvtx(name: str):
     return torch.cuda.nvtx.range(name)
 
 
-def partial_buffers(q_rows: int, n_h: int, d: int, n_parts: int, device="cuda"):
-    o = torch.empty((n_parts * q_rows, n_h, d), dtype=torch.float32, device=device)
+def partial_buffers(q_rows: int, n_h: int, d: int, n_parts: int, device="cuda", dtype=torch.float32):
+    o = torch.empty((n_parts * q_rows, n_h, d), dtype=dtype, device=device)
     lse = torch.empty((n_parts * q_rows, n_h), dtype=torch.float32, device=device)
     return o, lse
 
@@ -83,19 +83,32 @@ def run_ring(sched: RingSchedule, q, k, v, n_h: int, n_kv: int, out, lse_out=Non
     running (O, LSE) in its epilogue and the last step writes `out` directly
     (cp_attn_partial_fused; no merge pass). lse_out, if given, is the running
     LSE buffer.
+    merge="final_bf16": as "final" with bf16 partial O buffers
+    (cp_attn_partial_bf16_parts, then cp_attn_merge_bf16_parts): half the
+    partial bytes written and read.
     """
     q_rows, d = int(q.shape[0]), int(q.shape[-1])
     n = sched.n_ranks
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    n_bufs = n if merge == "final" else (1 if merge == "fused" else 2)
+    n_bufs = n if merge in ("final", "final_bf16") else (1 if merge == "fused" else 2)
     if o_parts is None:
-        o_parts, lse_parts = partial_buffers(q_rows, n_h, d, n_bufs, q.device)
+        o_parts, lse_parts = partial_buffers(q_rows, n_h, d, n_bufs, q.device,
+                                             torch.bfloat16 if merge == "final_bf16" else torch.float32)
     if workspace is None:
         workspace = torch.zeros(B.cp_workspace_size(B.CP_OP_PARTIAL, 0, n_h, d, 1), dtype=torch.uint8,
                                 device=q.device)
-    if merge not in ("fused", "final", "running"):
+    if merge not in ("fused", "final", "running", "final_bf16"):
         raise ValueError(merge)
+    if merge == "final_bf16":
+        for t in range(n):
+            blocks = sched.step_blocks(t, q_rows)
+            with _nvtx(f"ring step {t} (bf16 partials)"):
+                B.cp_attn_partial_bf16_parts(q, k, v, n_h, n_kv, scale, causal, sched.ranges, sched.n_ranges, blocks,
+                                             n, o_parts, lse_parts, workspace, stream)
+        with _nvtx(f"merge {n}-way (bf16 partials)"):
+            B.cp_attn_merge(o_parts, lse_parts, n, q_rows, q_rows, n_h, d, out, lse_out, stream)
+        return out
     if merge == "fused":
         lse_acc = lse_out if lse_out is not None else lse_parts
         for t in range(n):

@@ -248,6 +248,20 @@ cp_status cp_attn_partial_fused(const void* q, const void* k, const void* v, cp_
                                 int32_t n_blocks, float* o_acc, float* lse_acc, int64_t out_rows, int32_t accumulate,
                                 void* out, void* workspace, size_t ws_bytes, void* cuda_stream);
 
+/* cp_attn_partial writing its partial O rows in bf16 (round to nearest even)
+ * instead of fp32; the LSE stays fp32. A ring's partials then move half the
+ * bytes (the merge after the ring reads every partial once: method page,
+ * section 5, implementation detail 3), for about 2^-9 of relative rounding
+ * in each partial. Arguments as cp_attn_partial with o_part bf16
+ * [out_rows, n_h, d], 16-byte aligned. dtype CP_BF16 only (CP_ERR_UNSUPPORTED
+ * for CP_F32). Merge such partials with cp_attn_merge_bf16_parts. */
+cp_status cp_attn_partial_bf16_parts(const void* q, const void* k, const void* v, cp_dtype dtype,
+                                     int64_t q_rows, int64_t kv_rows, int32_t n_h, int32_t n_kv,
+                                     int32_t d, float softmax_scale, int32_t causal,
+                                     const cp_range* ranges, int32_t n_ranges, const cp_block* blocks,
+                                     int32_t n_blocks, void* o_part, float* lse_part, int64_t out_rows,
+                                     void* workspace, size_t ws_bytes, void* cuda_stream);
+
 /* LSE merge of n_parts partials of the same rows (method page, section 5,
  * implementation detail 3: the merge after pass-Q; the same step closes
  * pass-KV). Part j lives at o_parts + j*part_stride_rows*n_h*d and
@@ -263,6 +277,15 @@ cp_status cp_attn_partial_fused(const void* q, const void* k, const void* v, cp_
 cp_status cp_attn_merge(const float* o_parts, const float* lse_parts, int32_t n_parts,
                         int64_t part_stride_rows, int64_t rows, int32_t n_h, int32_t d, void* out,
                         cp_dtype out_dtype, float* lse_out, void* cuda_stream);
+
+/* cp_attn_merge of bf16 partials (as cp_attn_partial_bf16_parts writes them):
+ * o_parts bf16 at o_parts + j*part_stride_rows*n_h*d elements, 8-byte
+ * aligned; LSE parts fp32; the arithmetic is fp32 as in cp_attn_merge. out may
+ * be the same buffer as part 0 only with out_dtype CP_BF16 (CP_ERR_INVALID_ARG
+ * for an fp32 out on part 0). */
+cp_status cp_attn_merge_bf16_parts(const void* o_parts, const float* lse_parts, int32_t n_parts,
+                                   int64_t part_stride_rows, int64_t rows, int32_t n_h, int32_t d,
+                                   void* out, cp_dtype out_dtype, float* lse_out, void* cuda_stream);
 
 /* Split-KV decode (Flash Decoding; method page, section 5 software stack).
  * Request b has one query row q[b] at position L_b - 1 and keys k/v rows

@@ -48,8 +48,11 @@ def check(o_gpu, lse_gpu, o_ref, lse_ref, dtype: str, what: str = ""):
 
 
 def sample_rows(rng, n_rows: int, n_sample: int, must=()) -> np.ndarray:
+    """Sorted unique rows: every row of `must` plus seeded random others, at
+    least n_sample in all (or every row if there are fewer)."""
     must = np.unique(np.asarray([m for m in must if 0 <= m < n_rows], dtype=np.int64))
-    rest = rng.choice(n_rows, size=min(n_rows, max(0, n_sample - must.size)), replace=False)
+    others = np.setdiff1d(np.arange(n_rows, dtype=np.int64), must, assume_unique=True)
+    rest = rng.choice(others, size=min(others.size, max(0, n_sample - must.size)), replace=False)
     return np.unique(np.concatenate([must, rest]))
 
 

@@ -110,6 +110,21 @@ def test_bf16_ring(t, n_h, n_kv, n_ranks, variant, mode):
     _run_prefill(pr, n_ranks, variant, mode)
 
 
+@pytest.mark.parametrize("t,n_h,n_kv,n_ranks,variant,p,merge", [
+    (1000, 16, 1, 3, B.CP_PASS_KV, 0, "final"),
+    (777, 8, 2, 2, B.CP_PASS_Q, 0, "final"),
+    (300, 32, 2, 4, B.CP_PASS_Q, 1500, "final"),
+    (513, 128, 8, 2, B.CP_PASS_KV, 0, "fused"),
+    (129, 64, 1, 1, B.CP_PASS_KV, 0, "running"),
+])
+def test_bf16_ring_head_dim_64(t, n_h, n_kv, n_ranks, variant, p, merge):
+    """The tensor-core partial with D_H = 64 (its own instantiation: one
+    128-byte swizzle column per row, N = 64 PV products)."""
+    pr = synth.make_prefill(t, n_h, n_kv, 64, "bf16", 700 + t, 0.5, p=p)
+    _run_prefill(pr, n_ranks, variant, B.CP_SHARD_LOAD_BALANCED, merge=merge)
+    _run_prefill(pr, n_ranks, variant, B.CP_SHARD_LOAD_BALANCED, merge=merge, q_scale=8.0)
+
+
 @pytest.mark.parametrize("q_scale", [1.0, 8.0])
 def test_bf16_persistent_kv_pass_q(q_scale):
     """T new tokens over P cached + T keys, queries sharded and LSE-merged;
@@ -336,6 +351,40 @@ def test_bf16_ring_fused_merge(t, n_h, n_kv, n_ranks, variant, p):
     buffer, the last step writes bf16 out) equals unsharded attention."""
     pr = synth.make_prefill(t, n_h, n_kv, 128, "bf16", 200 + t, 0.5, p=p)
     _run_prefill(pr, n_ranks, variant, B.CP_SHARD_LOAD_BALANCED, merge="fused")
+
+
+@pytest.mark.parametrize("t,n_h,n_kv,n_ranks,variant,p,d", [
+    (1000, 16, 1, 3, B.CP_PASS_KV, 0, 128),
+    (300, 32, 2, 4, B.CP_PASS_Q, 1500, 128),
+    (777, 8, 2, 2, B.CP_PASS_KV, 0, 64),
+])
+def test_bf16_ring_bf16_partials(t, n_h, n_kv, n_ranks, variant, p, d):
+    """The ring with bf16 partial O buffers (cp_attn_partial_bf16_parts, then
+    cp_attn_merge_bf16_parts) equals unsharded attention within the bf16
+    tolerances, on diffuse and on peaked queries."""
+    pr = synth.make_prefill(t, n_h, n_kv, d, "bf16", 250 + t, 0.5, p=p)
+    _run_prefill(pr, n_ranks, variant, B.CP_SHARD_LOAD_BALANCED, merge="final_bf16")
+    _run_prefill(pr, n_ranks, variant, B.CP_SHARD_LOAD_BALANCED, merge="final_bf16", q_scale=8.0)
+
+
+@pytest.mark.parametrize("n_parts,out_dtype", [(2, "bf16"), (8, "f32"), (5, "bf16")])
+def test_merge_bf16_parts(n_parts, out_dtype):
+    """cp_attn_merge_bf16_parts on bf16 partials against the reference merge of
+    the same (rounded) values; -inf parts hold NaN and must not leak."""
+    rng = np.random.default_rng(200 + n_parts)
+    rows, n_h, d = 41, 4, 128
+    o = rng.standard_normal((n_parts, rows, n_h, d)).astype(np.float32)
+    lse = (rng.standard_normal((n_parts, rows, n_h)) * 3).astype(np.float32)
+    lse[rng.random(lse.shape) < 0.2] = -np.inf
+    o_bits = synth.bf16_bits(o)
+    o_vals = synth.bf16_bits_to_f32(o_bits)
+    o_ref, l_ref = OA.merge(list(np.where(np.isinf(lse)[..., None], 0.0, o_vals)), list(lse))
+    o_bits = np.where(np.isinf(lse)[..., None], np.uint16(0x7FC0), o_bits).astype(np.uint16)   # NaN in -inf parts
+    out = torch.empty((rows, n_h, d), dtype=torch.bfloat16 if out_dtype == "bf16" else torch.float32, device="cuda")
+    lse_out = torch.empty((rows, n_h), dtype=torch.float32, device="cuda")
+    B.cp_attn_merge(dev(o_bits, "bf16"), dev(lse, "f32"), n_parts, rows, rows, n_h, d, out, lse_out)
+    torch.cuda.synchronize()
+    check(out.float().cpu().numpy(), lse_out.cpu().numpy(), o_ref, l_ref, out_dtype, "merge of bf16 parts")
 
 
 def test_bf16_varlen_fused_merge():

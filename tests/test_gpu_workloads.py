@@ -68,10 +68,10 @@ def _gather(out, lse, rows):
     return out[sel].float().cpu().numpy(), lse[sel].cpu().numpy()
 
 
-@pytest.mark.parametrize("merge,q_mult", [("final", 1.0), ("fused", 1.0), ("final", 8.0)])
+@pytest.mark.parametrize("merge,q_mult", [("final", 1.0), ("fused", 1.0), ("final_bf16", 1.0), ("final", 8.0)])
 def test_prefill_128k_pass_kv(merge, q_mult):
-    """The headline step (separate 8-way merge), its fused-merge variant, and
-    the headline step on peaked queries."""
+    """The headline step (separate 8-way merge), its fused-merge and bf16-
+    partial variants, and the headline step on peaked queries."""
     w = synth.WORKLOADS["prefill_128k"]
     t, n_h, n_kv, d, n = w["t"], w["n_h"], w["n_kv"], w["d"], w["n_ranks"]
     q, k, v = _dev(w, synth.TENSOR_Q, t, n_h), _dev(w, synth.TENSOR_K, t, n_kv), _dev(w, synth.TENSOR_V, t, n_kv)
