@@ -79,6 +79,12 @@ struct Cfg {
   static constexpr int kSmemBytes = kSmemNeeded + 1024 <= kSmemMax ? kSmemNeeded + 1024 : kSmemMax;
   static_assert(kSmemNeeded <= kSmemMax, "shared memory plan exceeds 227 KB");
   static_assert(kKStages <= 3 && kVStages <= 3, "barrier slots hold at most 3 stages");
+  // Epilogue staging of a tile's output rows (fp32, rows padded by 16 bytes so
+  // that the per-row writes of a quarter warp hit distinct bank groups), over
+  // the Q and K regions, which no MMA or load touches any more by then.
+  static constexpr int kStageRow = HD * 4 + 16;
+  static constexpr int kStageTile = BM * kStageRow;
+  static_assert(kQTiles * kStageTile <= kOffV, "epilogue staging must stay clear of the V stages");
 };
 
 // barrier slots
@@ -525,7 +531,33 @@ __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Para
         lse_new = mx + logf(sum);
       }
     }
-    float* dst = p.o_part + out_idx * HD + hf * (HD / 2);
+    // The tile's rows go through shared memory so that global memory is read
+    // and written a whole row per warp instruction (a thread owns half a row;
+    // written straight from registers, every 32-byte sector would be touched
+    // half at a time by two instructions).
+    float* stage = reinterpret_cast<float*>(smem + x * C::kStageTile);   // [row][HD] + padding
+    const int wi = warp & 7;                       // warp within the tile's eight
+    const uint32_t tile_bar = 9 + x;               // named barrier of the tile's 256 softmax threads
+    done_ok = named_bar_and(tile_bar, 256, done_ok);
+    // global row of packed row r of this tile (for the copies; r's token must exist)
+    auto row_idx = [&](int r) -> int64_t {
+      const int tk = x * tok_per_tile + (r >> p.log2_group);
+      return (ws.out_row0 + q_row0 + tk) * p.n_h + kvh * group + (r & (group - 1));
+    };
+    constexpr int kRowsPerIns = 128 / HD;          // rows one warp instruction covers (float4 per lane)
+    constexpr int kLanesPerRow = 32 / kRowsPerIns;
+    if (done_ok && p.accumulate) {
+      // the earlier rows, a whole row per instruction, into the staging rows
+      for (int r0 = wi * 16; r0 < wi * 16 + 16; r0 += kRowsPerIns) {
+        const int r = r0 + lane / kLanesPerRow;
+        const int c4 = lane % kLanesPerRow;
+        if (x * tok_per_tile + (r >> p.log2_group) < n_tok)
+          *reinterpret_cast<float4*>(stage + r * (C::kStageRow / 4) + c4 * 4) =
+              *reinterpret_cast<const float4*>(p.o_part + row_idx(r) * HD + c4 * 4);
+      }
+    }
+    named_bar_sync(tile_bar, 256);
+    float* srow = stage + row * (C::kStageRow / 4) + hf * (HD / 2);   // this thread's half row
     if (done_ok) {
       if (n_iter > 0) tc_fence_after();
 #pragma unroll
@@ -545,25 +577,32 @@ __global__ void __maxnreg__(96) partial_bf16_kernel(const __grid_constant__ Para
           if (p.accumulate && wa != 0.0f) {   // an earlier row at -inf weighs 0 and is not read
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
-              const float4 pv = *reinterpret_cast<const float4*>(dst + c * 32 + i);
+              const float4 pv = *reinterpret_cast<const float4*>(srow + c * 32 + i);
               r[i] = fmaf(wa, pv.x, r[i]);
               r[i + 1] = fmaf(wa, pv.y, r[i + 1]);
               r[i + 2] = fmaf(wa, pv.z, r[i + 2]);
               r[i + 3] = fmaf(wa, pv.w, r[i + 3]);
             }
           }
-          if (p.out_final) {
-            uint4* fo = reinterpret_cast<uint4*>(p.out_final + out_idx * HD + hf * (HD / 2) + c * 32);
 #pragma unroll
-            for (int i = 0; i < 32; i += 8)
-              fo[i >> 3] = make_uint4(pack_bf16x2(r[i], r[i + 1]), pack_bf16x2(r[i + 2], r[i + 3]),
-                                      pack_bf16x2(r[i + 4], r[i + 5]), pack_bf16x2(r[i + 6], r[i + 7]));
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(dst + c * 32 + i) = make_float4(r[i], r[i + 1], r[i + 2], r[i + 3]);
-          }
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(srow + c * 32 + i) = make_float4(r[i], r[i + 1], r[i + 2], r[i + 3]);
         }
+      }
+    }
+    named_bar_sync(tile_bar, 256);
+    if (done_ok) {
+      // the tile's rows to global memory, a whole row per instruction
+      for (int r0 = wi * 16; r0 < wi * 16 + 16; r0 += kRowsPerIns) {
+        const int r = r0 + lane / kLanesPerRow;
+        const int c4 = lane % kLanesPerRow;
+        if (x * tok_per_tile + (r >> p.log2_group) >= n_tok) continue;
+        const float4 vv = *reinterpret_cast<const float4*>(stage + r * (C::kStageRow / 4) + c4 * 4);
+        if (p.out_final)
+          *reinterpret_cast<uint2*>(p.out_final + row_idx(r) * HD + c4 * 4) =
+              make_uint2(pack_bf16x2(vv.x, vv.y), pack_bf16x2(vv.z, vv.w));
+        else
+          *reinterpret_cast<float4*>(p.o_part + row_idx(r) * HD + c4 * 4) = vv;
       }
     }
     if (done_ok && row_valid && hf == 0) p.lse_part[out_idx] = lse_new;
