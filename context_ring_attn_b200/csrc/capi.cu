@@ -573,10 +573,24 @@ static cp_status merge_impl(const void* o_parts, cp_dtype parts_dtype, const flo
   grid = std::min<int64_t>(grid, 148 * 32);
   const unsigned g = static_cast<unsigned>(grid);
   const unsigned t = merge::kThreads;
-#define CP_MERGE_LAUNCH(InT, OutT, R_)                                                                         \
-  merge::merge_kernel<InT, OutT, R_><<<g, t, 0, stream>>>(static_cast<const InT*>(o_parts), lse_parts, n_parts,  \
-                                                          o_stride, l_stride, n_rowheads, d, static_cast<OutT*>(out), \
-                                                          lse_out)
+  // out on part 0 (or lse_out on LSE part 0): the in-place instantiation
+  const uintptr_t o_lo = reinterpret_cast<uintptr_t>(o_parts), o_hi = o_lo + static_cast<uintptr_t>(rows * n_h * d) *
+                                                                                  (parts_dtype == CP_F32 ? 4 : 2);
+  const uintptr_t ob = reinterpret_cast<uintptr_t>(out);
+  const uintptr_t l_lo = reinterpret_cast<uintptr_t>(lse_parts), l_hi = l_lo + static_cast<uintptr_t>(rows * n_h) * 4;
+  const uintptr_t lb = reinterpret_cast<uintptr_t>(lse_out);
+  const bool in_place = (ob >= o_lo && ob < o_hi) || (lse_out && lb >= l_lo && lb < l_hi);
+#define CP_MERGE_LAUNCH(InT, OutT, R_)                                                                              \
+  do {                                                                                                              \
+    if (in_place)                                                                                                   \
+      merge::merge_kernel_in_place<InT, OutT, R_><<<g, t, 0, stream>>>(                                           \
+          static_cast<const InT*>(o_parts), lse_parts, n_parts, o_stride, l_stride, n_rowheads, d,                \
+          static_cast<OutT*>(out), lse_out);                                                                        \
+    else                                                                                                            \
+      merge::merge_kernel<InT, OutT, R_><<<g, t, 0, stream>>>(static_cast<const InT*>(o_parts), lse_parts,       \
+                                                              n_parts, o_stride, l_stride, n_rowheads, d,         \
+                                                              static_cast<OutT*>(out), lse_out);                  \
+  } while (0)
 #define CP_MERGE_BY_R(InT, OutT)                \
   do {                                          \
     if (r == 1) CP_MERGE_LAUNCH(InT, OutT, 1);  \

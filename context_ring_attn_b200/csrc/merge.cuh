@@ -45,13 +45,13 @@ __device__ __forceinline__ void store4(__nv_bfloat16* dst, float4 v) {
   *reinterpret_cast<uint2*>(dst) = u;
 }
 
-// o_parts / lse_parts carry no __restrict__: out and lse_out may alias part 0.
 // InT: fp32 partials, or bf16 partial buffers (rounded O, fp32 LSE).
-template <typename InT, typename OutT, int R>
-__global__ void __launch_bounds__(kThreads, R <= 2 ? 3 : 2) merge_kernel(const InT* o_parts,
-                                                          const float* lse_parts, int n_parts,
-                                                          int64_t o_stride, int64_t l_stride, int64_t n_rowheads,
-                                                          int d, OutT* out, float* lse_out) {
+// kInPlace: out / lse_out may be part 0, so the part pointers carry no
+// __restrict__ promise; otherwise they do (the compiler may then schedule the
+// loads of a round freely around the stores).
+template <typename InT, typename OutT, int R, bool kInPlace>
+__device__ __forceinline__ void merge_body(const InT* o_parts, const float* lse_parts, int n_parts, int64_t o_stride,
+                                           int64_t l_stride, int64_t n_rowheads, int d, OutT* out, float* lse_out) {
   constexpr int C = kLoads / R;
   const int lane = threadIdx.x & 31;
   const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
@@ -132,6 +132,21 @@ __global__ void __launch_bounds__(kThreads, R <= 2 ? 3 : 2) merge_kernel(const I
         if (rh0 + r < n_rowheads) lse_out[rh0 + r] = lse_r[r];
     }
   }
+}
+
+template <typename InT, typename OutT, int R>
+__global__ void __launch_bounds__(kThreads, R <= 2 ? 3 : 2)
+    merge_kernel(const InT* __restrict__ o_parts, const float* __restrict__ lse_parts, int n_parts, int64_t o_stride,
+                 int64_t l_stride, int64_t n_rowheads, int d, OutT* __restrict__ out, float* __restrict__ lse_out) {
+  merge_body<InT, OutT, R, false>(o_parts, lse_parts, n_parts, o_stride, l_stride, n_rowheads, d, out, lse_out);
+}
+
+// out and lse_out may be part 0: no aliasing promise.
+template <typename InT, typename OutT, int R>
+__global__ void __launch_bounds__(kThreads, R <= 2 ? 3 : 2)
+    merge_kernel_in_place(const InT* o_parts, const float* lse_parts, int n_parts, int64_t o_stride,
+                          int64_t l_stride, int64_t n_rowheads, int d, OutT* out, float* lse_out) {
+  merge_body<InT, OutT, R, true>(o_parts, lse_parts, n_parts, o_stride, l_stride, n_rowheads, d, out, lse_out);
 }
 
 }  // namespace merge
