@@ -406,6 +406,7 @@ def run_ours(args, rank: int, world: int):
     if not args.no_secondary:
         for name in ("persistent_kv", "varlen_prefill"):
             secondary[name] = run_secondary(args, dev, name)
+        secondary["varlen_prefill_fused_merge"] = run_secondary(args, dev, "varlen_prefill", "fused")
         secondary["varlen_prefill_running_merge"] = run_secondary(args, dev, "varlen_prefill", "running")
 
     if rank != 0:
@@ -554,9 +555,10 @@ def run_secondary(args, dev, name: str, merge_override: str | None = None):
     """The other prefill workloads, each a full ring schedule per step:
     persistent-KV partial prefill (T=4096 new over P=126976 cached, 128/8
     heads, pass-Q, 8-way merge) and the varlen batch (8 sequences, 262144
-    tokens, 128/8 heads, pass-KV, merge fused into the partial kernel: its
-    partials are 17 GB per part, so the ring keeps one running buffer;
-    merge_override="running" times separate 2-way merges instead)."""
+    tokens, 128/8 heads, pass-KV; bf16 partial buffers, 8.6 GB per part, and
+    one 8-way merge; merge_override="fused" times the merge in the partial
+    kernel's epilogue with one fp32 running buffer, "running" separate 2-way
+    merges)."""
     import torch
 
     from context_ring_attn_b200 import binding as B
@@ -565,28 +567,34 @@ def run_secondary(args, dev, name: str, merge_override: str | None = None):
     w = synth.WORKLOADS[name]
     n_h, n_kv, d, n = w["n_h"], w["n_kv"], w["d"], w["n_ranks"]
     scale = 1.0 / math.sqrt(d)
+    shrink = max(1, args.shrink)   # profiling captures: every length divided by this (the mix kept)
     if name == "persistent_kv":
-        t, p = w["t"], w["p"]
+        t, p = w["t"] // shrink, w["p"] // shrink
         q_segs = [ring.Segment(t, 0, p, 0)]
         kv_segs = [ring.Segment(p, 0, 0, 0), ring.Segment(t, p, p, 0)]
         kv_rows, variant, merge = p + t, B.CP_PASS_Q, "final"
         desc = {"T": t, "P": p, "ring": "pass-Q", "merge": "final 8-way"}
     else:
-        lens = synth.varlen_lengths(w["seed"], w["n_seq"], w["total"])
-        t = w["total"]
+        lens = [ln // shrink for ln in synth.varlen_lengths(w["seed"], w["n_seq"], w["total"])]
+        t = sum(lens)
         starts = np.concatenate([[0], np.cumsum(lens)[:-1]]).astype(np.int64)
         q_segs = kv_segs = [ring.Segment(int(ln), int(s0), 0, i) for i, (ln, s0) in enumerate(zip(lens, starts))]
-        kv_rows, variant, merge = t, B.CP_PASS_KV, "fused"
+        kv_rows, variant, merge = t, B.CP_PASS_KV, "final_bf16"
         desc = {"seq_lens": [int(x) for x in lens], "ring": "pass-KV",
-                "merge": "fused into the partial kernel's epilogue (cp_attn_partial_fused), one running buffer"}
+                "merge": ("final 8-way over bf16 partial buffers (cp_attn_partial_bf16_parts, then "
+                          "cp_attn_merge_bf16_parts)")}
     if merge_override == "running":
         merge = "running"
         desc["merge"] = "running 2-way (cp_attn_merge after every step)"
+    elif merge_override == "fused":
+        merge = "fused"
+        desc["merge"] = "fused into the partial kernel's epilogue (cp_attn_partial_fused), one running buffer"
     q = synth.device_rows(w["seed"], synth.TENSOR_Q, t, (n_h, d), w["std"], "bf16", dev)
     k = synth.device_rows(w["seed"], synth.TENSOR_K, kv_rows, (n_kv, d), w["std"], "bf16", dev)
     v = synth.device_rows(w["seed"], synth.TENSOR_V, kv_rows, (n_kv, d), w["std"], "bf16", dev)
-    n_bufs = n if merge == "final" else (1 if merge == "fused" else 2)
-    o_parts, lse_parts = ring.partial_buffers(t, n_h, d, n_bufs, dev)
+    n_bufs = n if merge in ("final", "final_bf16") else (1 if merge == "fused" else 2)
+    o_parts, lse_parts = ring.partial_buffers(t, n_h, d, n_bufs, dev,
+                                              torch.bfloat16 if merge == "final_bf16" else torch.float32)
     out = torch.empty((t, n_h, d), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((t, n_h), dtype=torch.float32, device=dev)
     ws = torch.zeros(256, dtype=torch.uint8, device=dev)
@@ -599,7 +607,7 @@ def run_secondary(args, dev, name: str, merge_override: str | None = None):
     def step(record):
         sched = ring.RingSchedule(q_segs, kv_segs, n, variant)
         for s_ in range(n):
-            if merge == "final":
+            if merge in ("final", "final_bf16"):
                 target = lambda pt: pt
             elif merge == "fused":
                 target = lambda _pt: 0
@@ -612,6 +620,9 @@ def run_secondary(args, dev, name: str, merge_override: str | None = None):
             if merge == "fused":
                 B.cp_attn_partial_fused(q, k, v, n_h, n_kv, scale, True, sched.ranges, sched.n_ranges, blocks, n,
                                         o_parts, lse, s_ > 0, out if s_ == n - 1 else None, ws)
+            elif merge == "final_bf16":
+                B.cp_attn_partial_bf16_parts(q, k, v, n_h, n_kv, scale, True, sched.ranges, sched.n_ranges, blocks,
+                                             n, o_parts, lse_parts, ws)
             else:
                 B.cp_attn_partial(q, k, v, n_h, n_kv, scale, True, sched.ranges, sched.n_ranges, blocks, n,
                                   o_parts, lse_parts, ws)
@@ -628,16 +639,17 @@ def run_secondary(args, dev, name: str, merge_override: str | None = None):
                 if e:
                     e[1].record(stream)
                     ev_merge.append((e, 2 * t * n_h * (d + 1) * 4 + t * n_h * ((2 * d + 4) if last else (d + 1) * 4)))
-        if merge == "final":
+        if merge in ("final", "final_bf16"):
             e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) if record else None
             if e:
                 e[0].record(stream)
             B.cp_attn_merge(o_parts, lse_parts, n, t, t, n_h, d, out, lse)
             if e:
                 e[1].record(stream)
-                ev_merge.append((e, n * t * n_h * (d + 1) * 4 + t * n_h * (2 * d + 4)))
+                part_bytes = n * t * n_h * (d * (2 if merge == "final_bf16" else 4) + 4)
+                ev_merge.append((e, part_bytes + t * n_h * (2 * d + 4)))
 
-    for _ in range(3):
+    for _ in range(args.warmup):
         step(False)
     torch.cuda.synchronize()
     steps = max(2, args.steps // 4)
@@ -908,6 +920,12 @@ def main():
     ap.add_argument("--no-fused", action="store_true", help="skip timing the fused-merge variant of the step")
     ap.add_argument("--no-secondary", action="store_true", help="skip the persistent-KV and varlen workloads")
     ap.add_argument("--only-decode", action="store_true", help="time the split-KV decode workload alone")
+    ap.add_argument("--only-workload", choices=["persistent_kv", "varlen_prefill"], default=None,
+                    help="time one of the other prefill workloads alone (prints its own line)")
+    ap.add_argument("--merge", choices=["fused", "running"], default=None,
+                    help="with --only-workload varlen_prefill: the merge mode")
+    ap.add_argument("--shrink", type=int, default=1,
+                    help="with --only-workload: divide every length by this (smaller profiling captures)")
     ap.add_argument("--sweep-miss-rate", action="store_true",
                     help="Algorithm 1 sweep of pass-KV vs pass-Q over KV-cache miss rates (prints its own line)")
     ap.add_argument("--tokens", type=int, default=0,
@@ -932,6 +950,10 @@ def main():
     try:
         if args.only_decode:
             print(json.dumps({"decode": run_decode(args, torch.device("cuda", local))}), flush=True)
+            return
+        if args.only_workload:
+            res = run_secondary(args, torch.device("cuda", local), args.only_workload, args.merge)
+            print(json.dumps({args.only_workload: res, "shrink": args.shrink}), flush=True)
             return
         if args.sweep_miss_rate:
             if rank == 0:

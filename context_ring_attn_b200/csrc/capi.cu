@@ -619,9 +619,41 @@ cp_status cp_attn_merge(const float* o_parts, const float* lse_parts, int32_t n_
 cp_status cp_attn_merge_bf16_parts(const void* o_parts, const float* lse_parts, int32_t n_parts,
                                    int64_t part_stride_rows, int64_t rows, int32_t n_h, int32_t d, void* out,
                                    cp_dtype out_dtype, float* lse_out, void* cuda_stream) {
-  if (out == o_parts && out_dtype == CP_F32) return CP_ERR_INVALID_ARG;   // in place needs matching element sizes
-  return merge_impl(o_parts, CP_BF16, lse_parts, n_parts, part_stride_rows, rows, n_h, d, out, out_dtype, lse_out,
-                    cuda_stream);
+  if (!o_parts || !lse_parts || !out) return CP_ERR_INVALID_ARG;
+  if (n_parts < 1 || rows < 0 || n_h < 1 || d < 8 || (d & 7) || d > 256) return CP_ERR_INVALID_ARG;
+  if (n_parts > 1 && part_stride_rows < rows) return CP_ERR_INVALID_ARG;
+  if (!aligned(o_parts, 16) || !aligned(lse_parts, 4)) return CP_ERR_INVALID_ARG;
+  if (out_dtype == CP_F32) {
+    if (!aligned(out, 16)) return CP_ERR_INVALID_ARG;
+  } else if (out_dtype == CP_BF16) {
+    if (!aligned(out, 8)) return CP_ERR_INVALID_ARG;
+  } else {
+    return CP_ERR_UNSUPPORTED;
+  }
+  // out and lse_out may not overlap the parts (rows are read and written by different lanes)
+  const uintptr_t o_lo = reinterpret_cast<uintptr_t>(o_parts);
+  const uintptr_t o_hi = o_lo + static_cast<uintptr_t>((n_parts > 1 ? (n_parts - 1) * part_stride_rows : 0) + rows) *
+                                    n_h * d * 2;
+  const uintptr_t ob = reinterpret_cast<uintptr_t>(out);
+  const uintptr_t oe = ob + static_cast<uintptr_t>(rows) * n_h * d * (out_dtype == CP_F32 ? 4 : 2);
+  if (rows > 0 && ob < o_hi && oe > o_lo) return CP_ERR_INVALID_ARG;
+  const int64_t n_rowheads = rows * n_h;
+  if (n_rowheads == 0) return CP_OK;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  const int64_t rows_per_warp = 32 / (d / 8);
+  const int64_t warps_per_block = merge::kThreads / 32;
+  int64_t grid = (n_rowheads + warps_per_block * rows_per_warp - 1) / (warps_per_block * rows_per_warp);
+  grid = std::min<int64_t>(grid, 148 * 32);
+  const int64_t o_stride = part_stride_rows * n_h * d, l_stride = part_stride_rows * n_h;
+  if (out_dtype == CP_F32)
+    merge::merge_bf16_parts_kernel<float><<<static_cast<unsigned>(grid), merge::kThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o_parts), lse_parts, n_parts, o_stride, l_stride, n_rowheads, d,
+        static_cast<float*>(out), lse_out);
+  else
+    merge::merge_bf16_parts_kernel<__nv_bfloat16><<<static_cast<unsigned>(grid), merge::kThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o_parts), lse_parts, n_parts, o_stride, l_stride, n_rowheads, d,
+        static_cast<__nv_bfloat16*>(out), lse_out);
+  return last_cuda_status();
 }
 
 static cp_status decode_impl(const void* q, const void* k, const void* v, cp_dtype dtype, const int64_t* kv_offsets,

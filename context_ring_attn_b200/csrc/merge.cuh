@@ -149,5 +149,81 @@ __global__ void __launch_bounds__(kThreads, R <= 2 ? 3 : 2)
   merge_body<InT, OutT, R, true>(o_parts, lse_parts, n_parts, o_stride, l_stride, n_rowheads, d, out, lse_out);
 }
 
+// The same merge over bf16 partial buffers. A lane loads 8 bf16 (16 bytes) of
+// a part per round, so one row-head of D columns takes D/8 lanes and a warp
+// covers 32*8/D row-heads at a time; each round brings 8 parts of every
+// row-head (as many bytes in flight per lane as the fp32 kernel). Needs
+// D % 8 == 0 and D <= 256; out may not alias the parts.
+constexpr int kMergeParts16 = 8;
+
+__device__ __forceinline__ void unpack8(const uint4 u, float (&f)[8]) {
+  f[0] = __uint_as_float(u.x << 16); f[1] = __uint_as_float(u.x & 0xffff0000u);
+  f[2] = __uint_as_float(u.y << 16); f[3] = __uint_as_float(u.y & 0xffff0000u);
+  f[4] = __uint_as_float(u.z << 16); f[5] = __uint_as_float(u.z & 0xffff0000u);
+  f[6] = __uint_as_float(u.w << 16); f[7] = __uint_as_float(u.w & 0xffff0000u);
+}
+
+template <typename OutT>
+__global__ void __launch_bounds__(kThreads, 2)
+    merge_bf16_parts_kernel(const __nv_bfloat16* __restrict__ o_parts, const float* __restrict__ lse_parts,
+                            int n_parts, int64_t o_stride, int64_t l_stride, int64_t n_rowheads, int d,
+                            OutT* __restrict__ out, float* __restrict__ lse_out) {
+  const int lane = threadIdx.x & 31;
+  const int lanes_per_row = d >> 3;                 // 8 columns per lane
+  const int rows_per_warp = 32 / lanes_per_row;
+  const int sub = lane / lanes_per_row;             // row-head of this lane within the warp's group
+  const int vi = lane - sub * lanes_per_row;        // its 8-column slice
+  const bool active = sub < rows_per_warp;
+  const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
+  for (int64_t rh0 = warp_global * rows_per_warp; rh0 < n_rowheads; rh0 += n_warps * rows_per_warp) {
+    const int64_t rh = rh0 + sub;
+    const bool mine = active && rh < n_rowheads;
+    float m = -INFINITY, l = 0.0f;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int jb = 0; jb < n_parts; jb += kMergeParts16) {
+      float lj[kMergeParts16];
+      uint4 x[kMergeParts16];
+#pragma unroll
+      for (int c = 0; c < kMergeParts16; ++c) {
+        const int j = jb + c;
+        lj[c] = -INFINITY;
+        x[c] = make_uint4(0u, 0u, 0u, 0u);
+        if (mine && j < n_parts) {
+          lj[c] = lse_parts[j * l_stride + rh];
+          x[c] = __ldcs(reinterpret_cast<const uint4*>(o_parts + j * o_stride + rh * d) + vi);
+        }
+      }
+      float mx = lj[0];
+#pragma unroll
+      for (int c = 1; c < kMergeParts16; ++c) mx = fmaxf(mx, lj[c]);
+      const float m_new = fmaxf(m, mx);
+      const float mu = (m_new == -INFINITY) ? 0.0f : m_new;   // parts at -inf weigh 0
+      const float sc = expf(m - mu);
+      l *= sc;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] *= sc;
+#pragma unroll
+      for (int c = 0; c < kMergeParts16; ++c) {
+        if (lj[c] == -INFINITY) continue;   // its O row is not used (it may hold anything)
+        const float w = expf(lj[c] - mu);
+        float f[8];
+        unpack8(x[c], f);
+        l += w;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, f[i], acc[i]);
+      }
+      m = m_new;
+    }
+    if (mine) {
+      const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
+      OutT* dst = out + rh * d + vi * 8;
+      store4(dst, make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv));
+      store4(dst + 4, make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv));
+      if (lse_out && vi == 0) lse_out[rh] = (l > 0.0f) ? m + logf(l) : -INFINITY;
+    }
+  }
+}
+
 }  // namespace merge
 }  // namespace cpk

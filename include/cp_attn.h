@@ -279,10 +279,10 @@ cp_status cp_attn_merge(const float* o_parts, const float* lse_parts, int32_t n_
                         cp_dtype out_dtype, float* lse_out, void* cuda_stream);
 
 /* cp_attn_merge of bf16 partials (as cp_attn_partial_bf16_parts writes them):
- * o_parts bf16 at o_parts + j*part_stride_rows*n_h*d elements, 8-byte
- * aligned; LSE parts fp32; the arithmetic is fp32 as in cp_attn_merge. out may
- * be the same buffer as part 0 only with out_dtype CP_BF16 (CP_ERR_INVALID_ARG
- * for an fp32 out on part 0). */
+ * o_parts bf16 at o_parts + j*part_stride_rows*n_h*d elements, 16-byte
+ * aligned; LSE parts fp32; the arithmetic is fp32 as in cp_attn_merge.
+ * Needs d % 8 == 0 and d <= 256; out may not overlap the parts
+ * (CP_ERR_INVALID_ARG otherwise). */
 cp_status cp_attn_merge_bf16_parts(const void* o_parts, const float* lse_parts, int32_t n_parts,
                                    int64_t part_stride_rows, int64_t rows, int32_t n_h, int32_t d,
                                    void* out, cp_dtype out_dtype, float* lse_out, void* cuda_stream);

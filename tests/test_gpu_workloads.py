@@ -151,10 +151,12 @@ def test_decode_split_full():
     check(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "bf16", "decode_split")
 
 
-@pytest.mark.parametrize("merge,q_mult", [("fused", 1.0), ("running", 1.0), ("fused", 8.0)])
+@pytest.mark.parametrize("merge,q_mult", [("final_bf16", 1.0), ("fused", 1.0), ("running", 1.0),
+                                          ("final_bf16", 8.0)])
 def test_varlen_prefill_pass_kv(merge, q_mult):
-    """The full varlen workload in both merge modes the bench times (fused is
-    the workload's default), and the default on peaked queries."""
+    """The full varlen workload in the merge modes the bench times (bf16
+    partial buffers and one 8-way merge is the workload's default), and the
+    default on peaked queries."""
     w = synth.WORKLOADS["varlen_prefill"]
     lens = synth.varlen_lengths(w["seed"], w["n_seq"], w["total"])
     total, n_h, n_kv, d, n = w["total"], w["n_h"], w["n_kv"], w["d"], w["n_ranks"]
@@ -172,7 +174,7 @@ def test_varlen_prefill_pass_kv(merge, q_mult):
     B.cp_check_status(ws)
     must = [int(s) for s in starts] + [int(s + ln - 1) for s, ln in zip(starts, lens)]
     must += _chunk_edges([int(x) for x in lens], [int(s) for s in starts], n)
-    n_sample = N_SAMPLE if (merge, q_mult) == ("fused", 1.0) else N_SAMPLE_VARIANT
+    n_sample = N_SAMPLE if (merge, q_mult) == ("final_bf16", 1.0) else N_SAMPLE_VARIANT
     rows = sample_rows(np.random.default_rng(5 + int(q_mult)), total, n_sample, must)
     assert rows.size >= n_sample
     o_gpu, l_gpu = _gather(out, lse, rows)
