@@ -400,10 +400,14 @@ def run_ours(args, rank: int, world: int):
 
     e2e = run_e2e(args, q, k, v, out, lse, o_parts, lse_parts, ws, segs, n_ranks, n_h, n_kv, world, dev,
                   step_flops, barrier) if not args.no_e2e else None
-    decode = run_decode(args, dev) if not args.no_decode else None
-    context = run_library_context(args, dev) if not args.no_context else None
+    # The other workloads, the library context and the CPU baseline are
+    # measured at N = 1 only: with N > 1 every rank would repeat the same
+    # single-GPU figures while all N GPUs are held.
+    single = world == 1
+    decode = run_decode(args, dev) if single and not args.no_decode else None
+    context = run_library_context(args, dev) if single and not args.no_context else None
     secondary = {}
-    if not args.no_secondary:
+    if single and not args.no_secondary:
         for name in ("persistent_kv", "varlen_prefill"):
             secondary[name] = run_secondary(args, dev, name)
         secondary["varlen_prefill_fused_merge"] = run_secondary(args, dev, "varlen_prefill", "fused")
@@ -449,7 +453,9 @@ def run_ours(args, rank: int, world: int):
         line["library_context"] = context
     if secondary:
         line["workloads"] = secondary
-    if not args.no_cpu_baseline:
+    if not single:
+        line["secondary_legs"] = "decode, other workloads, library context and cpu_baseline are measured at N=1 only"
+    if single and not args.no_cpu_baseline:
         f, s, n = oracle_sample(0.0, seed=0, min_runs=args.cpu_rows // ORACLE_RUN)
         rate = f / s
         line["cpu_baseline"] = {
