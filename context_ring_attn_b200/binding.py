@@ -135,8 +135,9 @@ def _ptr(t) -> int | None:
 
 
 def _stream(stream) -> int | None:
+    """A raw cudaStream_t handle, or a torch.cuda.Stream; None: torch's current stream."""
     if stream is not None:
-        return int(stream)
+        return int(getattr(stream, "cuda_stream", stream))
     import torch
     return int(torch.cuda.current_stream().cuda_stream)
 
