@@ -201,14 +201,14 @@ constexpr size_t kStatusBytes = 256;
 inline size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Ranges of the flattened decode keys (one per warp of the persistent split
-// grid): 8 per SM of the current device, at most n_splits per flattened
+// grid): dec::kWarps per SM of the current device, at most n_splits per flattened
 // (request, KV head, unit) triple.
 cp_status decode_ranges(int32_t n_splits, int32_t batch, int32_t triples_per_request, int32_t* n_warps) {
   int n_sm = 0, dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return CP_ERR_CUDA;
-  const int64_t want = (static_cast<int64_t>(n_splits) * batch * triples_per_request + 7) / 8;
-  *n_warps = static_cast<int32_t>(std::max<int64_t>(1, std::min<int64_t>(n_sm, want)) * 8);
+  const int64_t want = (static_cast<int64_t>(n_splits) * batch * triples_per_request + dec::kWarps - 1) / dec::kWarps;
+  *n_warps = static_cast<int32_t>(std::max<int64_t>(1, std::min<int64_t>(n_sm, want)) * dec::kWarps);
   return CP_OK;
 }
 
