@@ -165,13 +165,16 @@ def test_gqa_head_grouping_matches_page(golden):
 @pytest.mark.parametrize("n_ranks", [1, 2, 3, 4])
 @pytest.mark.parametrize("mode", [P.LOAD_BALANCED, P.CONTIGUOUS])
 @pytest.mark.parametrize("variant", [P.PASS_KV, P.PASS_Q])
-def test_shard_and_merge_equals_unsharded(n_ranks, mode, variant):
+@pytest.mark.parametrize("group", [1, 2, 4])
+def test_shard_and_merge_equals_unsharded(n_ranks, mode, variant, group):
     """The ring is lossless exact: any plan, ring variant and merge order gives
-    the unsharded result (method page, section 2 and section 4)."""
-    rng = np.random.default_rng(100 * n_ranks + 10 * mode + variant)
+    the unsharded result (method page, section 2 and section 4), for GQA groups
+    of 1, 2 and 4 query heads per KV head."""
+    rng = np.random.default_rng(1000 * group + 100 * n_ranks + 10 * mode + variant)
     lens = [29, 16]
     tot = sum(lens)
-    n_h, n_kv, d = 4, 2, 8
+    n_h, d = 4, 8
+    n_kv = n_h // group
     q, k, v = _rand(rng, tot, n_h, d), _rand(rng, tot, n_kv, d), _rand(rng, tot, n_kv, d)
     seq = np.repeat(np.arange(len(lens)), lens)
     pos = np.concatenate([np.arange(n) for n in lens])
