@@ -3,9 +3,9 @@ every dimension the hot path takes (sequence lengths including ragged and
 one-token ones, cached prefixes, several sequences, rank counts, GQA group
 sizes, head dims, ring variant, shard mode, merge mode, peaked queries), each
 run through the library and checked against the fp64 reference with the bf16
-tolerances of the other tests; and the same for split-KV decode (request
-counts, lengths including 0 and 1, groups up to 64 heads, head dims, split
-counts). The draws are fixed by the case index, so a failure names a
+tolerances of the other tests (the exact fp32 path at 1e-5); and the same
+for split-KV decode (request counts, lengths including 0 and 1, groups up to
+64 heads, head dims, split counts). The draws are fixed by the case index, so a failure names a
 reproducible configuration."""
 import math
 
@@ -23,6 +23,7 @@ from test_gpu_kernels import _run_prefill
 pytestmark = pytest.mark.gpu
 
 N_RING = 96
+N_EXACT = 24
 N_DECODE = 48
 
 
@@ -65,6 +66,25 @@ def test_random_ring(i):
             segs.append(ring.Segment(n, r0, 0, s))
             r0 += n
     _run_prefill(pr, c["n_ranks"], c["variant"], c["mode"], merge=c["merge"], q_scale=c["q_scale"], segs=segs)
+
+
+def _exact_case(i):
+    rng = np.random.default_rng(7170 + i)
+    group = int(rng.choice([1, 2, 4, 8]))
+    n_kv = int(rng.choice([1, 2]))
+    return dict(d=int(rng.choice([64, 128])), n_h=group * n_kv, n_kv=n_kv,
+                variant=int(rng.choice([B.CP_PASS_KV, B.CP_PASS_Q])),
+                mode=int(rng.choice([B.CP_SHARD_LOAD_BALANCED, B.CP_SHARD_CONTIGUOUS])),
+                n_ranks=int(rng.integers(1, 6)), merge=str(rng.choice(["final", "running"])),
+                t=int(rng.integers(1, 200)), p=int(rng.integers(1, 300)) if rng.random() < 0.4 else 0)
+
+
+@pytest.mark.parametrize("i", range(N_EXACT))
+def test_random_exact_fp32(i):
+    """The exact fp32 path at its 1e-5 tolerance."""
+    c = _exact_case(i)
+    pr = synth.make_prefill(c["t"], c["n_h"], c["n_kv"], c["d"], "f32", 9700 + i, 1.0, p=c["p"])
+    _run_prefill(pr, c["n_ranks"], c["variant"], c["mode"], merge=c["merge"])
 
 
 def _decode_case(i):
