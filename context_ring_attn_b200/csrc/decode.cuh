@@ -193,9 +193,10 @@ struct Walker {
   }
 };
 
-// Let the merge launch (a programmatic dependent of this grid) start its
-// blocks early: they wait in griddepcontrol.wait until this grid has finished
-// and its writes are visible, so the launch gap is hidden.
+// Let the merge launch (a programmatic dependent of this grid) proceed while
+// this grid runs: its blocks are placed as SMs free up and wait in
+// griddepcontrol.wait until this grid has finished and its writes are
+// visible, so no launch gap separates the two kernels.
 __device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
