@@ -103,3 +103,16 @@ def test_ring_covers_every_pair_once(n, variant):
             assert kr[0] == i and qr[0] == (i - t) % n
     assert seen == set(itertools.product(range(n), range(n)))
     assert all(sorted(v) == list(range(n)) for v in per_q_parts.values())
+
+
+@pytest.mark.parametrize("k", [1000, 1024])
+def test_contiguous_layout_matches_page(golden, k):
+    """The contiguous shard mode is the layout the CP/EP page prints for 128K
+    tokens on 8 GPUs (GPU r holds tokens 16K*r .. 16K*(r+1)); K is read as
+    1000 and as 1024 tokens, and the layout holds for both."""
+    seq_k, n = (int(x) for x in golden["cp_layout_sequence_k_and_ranks"])
+    first = [int(x) * k for x in golden["cp_layout_rank_first_token_k"]]
+    segs = [P.Segment(seq_k * k, 0, 0, 0)]
+    for r in range(n):
+        rows = [t for g in P.rank_ranges(segs, n, P.CONTIGUOUS, r) for t in range(g.row0, g.row0 + g.length)]
+        assert rows == list(range(first[r], first[r + 1]))

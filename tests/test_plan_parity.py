@@ -173,3 +173,16 @@ def test_select_ring_variant_matches_oracle():
         B.cp_select_ring_variant(0, 0, 128, 8, 128, 8, 2, 50e9, 0.0)
     with pytest.raises(B.CpError):
         B.cp_select_ring_variant(10, 10, 128, 8, 128, 8, 2, 0.0, 0.0)
+
+
+@pytest.mark.parametrize("k", [1000, 1024])
+def test_library_contiguous_layout_matches_page(golden, k):
+    """cp_rank_ranges in contiguous mode gives GPU r the tokens the CP/EP page
+    prints for 128K tokens on 8 GPUs: 16K*r .. 16K*(r+1)."""
+    seq_k, n = (int(x) for x in golden["cp_layout_sequence_k_and_ranks"])
+    first = [int(x) * k for x in golden["cp_layout_rank_first_token_k"]]
+    segs = B.segments([(seq_k * k, 0, 0, 0)])
+    for r in range(n):
+        got = B.cp_rank_ranges(segs, 1, n, B.CP_SHARD_CONTIGUOUS, r)
+        rows = [t for g in got for t in range(g.row0, g.row0 + g.len)]
+        assert rows == list(range(first[r], first[r + 1]))
