@@ -5,14 +5,24 @@ the load-balanced shard plan for 8 virtual ranks (host), the 8 pass-KV ring
 steps (one cp_attn_partial launch each, tcgen05 kernel) and the 8-way LSE
 merge into the bf16 output. Workload: Llama3-405B per-TP8-rank head slice,
 N_H=16, N_KV=1, D_H=128, T=131072, bf16 inputs iid N(0,1)*0.5 (seeded,
-synthetic). The split-KV decode workload (32 requests, 256 splits) is timed
-in the same run and reported under "decode".
+synthetic). Inputs are resident in HBM and larger than L2 (no flush).
+Beside the headline the same line reports: the roofline of the partial
+kernel (per-launch CUDA events) with the DRAM traffic of the committed ncu
+capture, the step with the merge fused into the partial kernel and with bf16
+partial buffers, the step end to end from pinned host memory ("e2e"), the
+split-KV decode workload (32 requests, 256 splits), the persistent-KV and
+varlen workloads, cuDNN's fused attention on the same inputs (context only),
+SM clocks sampled during the timed region, and the fp64 reference timed on
+the host's cores on a sample of rows ("cpu_baseline").
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 N > 1 (launched by torchrun): every rank runs its own copy of the workload
 (independent replicas, weak scaling, no data-path collective); the time is
-the max over ranks and `value` counts the work of all ranks.
+the max over ranks and `value` counts the work of all ranks; the other
+workloads, the context figure and the CPU baseline are measured at N = 1 only.
+--impl reference times the fp64 reference (the host's cores) on the same
+metric and configuration.
 """
 from __future__ import annotations
 
