@@ -163,8 +163,10 @@ __device__ __forceinline__ void unpack8(const uint4 u, float (&f)[8]) {
   f[6] = __uint_as_float(u.w << 16); f[7] = __uint_as_float(u.w & 0xffff0000u);
 }
 
+// Three CTAs per SM (at most 85 registers a thread; 76 used, no spills): more
+// loads in flight than two, +5% measured on an 8-way merge of bf16 parts.
 template <typename OutT>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 3)
     merge_bf16_parts_kernel(const __nv_bfloat16* __restrict__ o_parts, const float* __restrict__ lse_parts,
                             int n_parts, int64_t o_stride, int64_t l_stride, int64_t n_rowheads, int d,
                             OutT* __restrict__ out, float* __restrict__ lse_out) {
